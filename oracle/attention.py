@@ -1,0 +1,177 @@
+"""Masked softmax attention, forward and backward -- plain CPU reference, fp64.
+
+TEST INFRASTRUCTURE ONLY (see the package docstring): never imported by the
+product path.
+
+The method computes exactly (up to rounding order) the masked softmax
+attention of [review] §3 Eq.2, ``O = softmax(Q K^T * scale + M) V`` with
+``M`` = 0 on allowed pairs and -inf elsewhere; its block-sparse execution
+([review] §4.2, 128x128 blocks) only skips tiles where ``M`` is -inf
+everywhere.  So this module is that definition written out, with no blocking,
+fusion or reordering.  The pages fix neither the scale nor the saved
+statistics; the readings taken: ``scale = 1/sqrt(d)`` (the Eq.1 convention),
+``LSE`` = natural-log log-sum-exp of the masked, scaled logits per row.
+
+Backward ([review] §4.3 uses the same attention under LoRA fine-tuning, so
+its gradients are needed; the pages print no formulas): the plain
+derivative of Eq.2 --
+    P  = exp(S - LSE)                (S masked to -inf off the mask)
+    dV = P^T dO
+    dP = dO V^T
+    Dr = rowsum(dO * O)
+    dS = P * (dP - Dr)
+    dQ = scale * dS K,   dK = scale * dS^T Q.
+
+Every array is float64; callers pass bf16-rounded values where the device
+consumes bf16 (the oracle then sees exactly the device's inputs).
+"""
+
+from __future__ import annotations
+
+import numpy as np
+
+from . import mask as _mask
+
+
+def _as64(x):
+    return np.asarray(x, dtype=np.float64)
+
+
+def forward(q, k, v, allowed, scale):
+    """[review] §3 Eq.2 for one (batch, head): q,k,v (n, d); allowed (n, n) bool.
+
+    Returns (O (n, d), LSE (n,)).  A row with no allowed key gets O = 0,
+    LSE = -inf (cannot happen under the radial mask: same-frame is dense).
+    """
+    q, k, v = _as64(q), _as64(k), _as64(v)
+    S = (q @ k.T) * scale
+    S = np.where(allowed, S, -np.inf)
+    m = S.max(axis=1, keepdims=True)
+    live = np.isfinite(m)
+    m0 = np.where(live, m, 0.0)
+    P = np.exp(S - m0)
+    l = P.sum(axis=1, keepdims=True)
+    with np.errstate(divide="ignore", invalid="ignore"):
+        O = np.where(live, (P / np.where(live, l, 1.0)) @ v, 0.0)
+        lse = np.where(live[:, 0], m0[:, 0] + np.log(np.where(live[:, 0], l[:, 0], 1.0)), -np.inf)
+    return O, lse
+
+
+def backward(q, k, v, o, do, lse, allowed, scale):
+    """Gradients of Eq.2 for one (batch, head).  Returns (dQ, dK, dV)."""
+    q, k, v, o, do, lse = (_as64(x) for x in (q, k, v, o, do, lse))
+    S = (q @ k.T) * scale
+    with np.errstate(invalid="ignore"):
+        P = np.where(allowed, np.exp(S - lse[:, None]), 0.0)
+    dV = P.T @ do
+    dP = do @ v.T
+    Dr = (do * o).sum(axis=1)
+    dS = P * (dP - Dr[:, None])
+    dQ = scale * (dS @ k)
+    dK = scale * (dS.T @ q)
+    return dQ, dK, dV
+
+
+# ---------------------------------------------------------------------------
+# Radial-mask wrappers over [B, H, N, D] arrays
+# ---------------------------------------------------------------------------
+
+def radial_forward(q, k, v, f, s, sink=True, scale=None):
+    """Eq.2 under the radial mask for every (batch, head) of [B, H, N, D] inputs."""
+    q, k, v = _as64(q), _as64(k), _as64(v)
+    Bn, H, N, D = q.shape
+    assert N == f * s
+    scale = 1.0 / np.sqrt(D) if scale is None else scale
+    M = _mask.token_mask(f, s, sink)
+    O = np.empty_like(q)
+    L = np.empty((Bn, H, N))
+    for b in range(Bn):
+        for h in range(H):
+            O[b, h], L[b, h] = forward(q[b, h], k[b, h], v[b, h], M, scale)
+    return O, L
+
+
+def radial_backward(q, k, v, o, do, lse, f, s, sink=True, scale=None):
+    """Gradients under the radial mask for every (batch, head)."""
+    q = _as64(q)
+    Bn, H, N, D = q.shape
+    scale = 1.0 / np.sqrt(D) if scale is None else scale
+    M = _mask.token_mask(f, s, sink)
+    out = [np.empty_like(q) for _ in range(3)]
+    for b in range(Bn):
+        for h in range(H):
+            g = backward(q[b, h], k[b, h], v[b, h], o[b, h], do[b, h], lse[b, h], M, scale)
+            for t in range(3):
+                out[t][b, h] = g[t]
+    return tuple(out)
+
+
+# ---------------------------------------------------------------------------
+# Row-sampled evaluation (large shapes: each output row computed on its own)
+# ---------------------------------------------------------------------------
+
+def forward_rows(q, k, v, rows, f, s, sink=True, scale=None, chunk=256):
+    """O and LSE of the given query rows of one (batch, head): q,k,v (n, d).
+
+    Row r only needs its own logits against all keys, so it is Eq.2 applied to
+    those rows alone.  Returns (O_rows (R, d), LSE_rows (R,)).
+    """
+    q, k, v = _as64(q), _as64(k), _as64(v)
+    rows = np.asarray(rows, dtype=np.int64)
+    scale = 1.0 / np.sqrt(q.shape[1]) if scale is None else scale
+    O = np.empty((rows.size, q.shape[1]))
+    L = np.empty(rows.size)
+    for c0 in range(0, rows.size, chunk):
+        r = rows[c0:c0 + chunk]
+        M = _mask.row_mask(r, f, s, sink)
+        S = (q[r] @ k.T) * scale
+        S = np.where(M, S, -np.inf)
+        m = S.max(axis=1, keepdims=True)
+        P = np.exp(S - m)
+        l = P.sum(axis=1, keepdims=True)
+        O[c0:c0 + r.size] = (P / l) @ v
+        L[c0:c0 + r.size] = m[:, 0] + np.log(l[:, 0])
+    return O, L
+
+
+def dq_rows(q, k, v, do, rows, f, s, sink=True, scale=None, chunk=256):
+    """dQ of the given query rows of one (batch, head).
+
+    dQ_r depends only on row r's own logits, its O_r, LSE_r and dO_r, all of
+    which are recomputed here in fp64 from the inputs.
+    """
+    q, k, v, do = _as64(q), _as64(k), _as64(v), _as64(do)
+    rows = np.asarray(rows, dtype=np.int64)
+    scale = 1.0 / np.sqrt(q.shape[1]) if scale is None else scale
+    out = np.empty((rows.size, q.shape[1]))
+    for c0 in range(0, rows.size, chunk):
+        r = rows[c0:c0 + chunk]
+        M = _mask.row_mask(r, f, s, sink)
+        S = np.where(M, (q[r] @ k.T) * scale, -np.inf)
+        m = S.max(axis=1, keepdims=True)
+        P = np.exp(S - m)
+        P /= P.sum(axis=1, keepdims=True)
+        o = P @ v
+        dP = do[r] @ v.T
+        Dr = (do[r] * o).sum(axis=1)
+        dS = P * (dP - Dr[:, None])
+        out[c0:c0 + r.size] = scale * (dS @ k)
+    return out
+
+
+def sample_rows(n, count, s, B, seed):
+    """Seeded sample of query rows: first/last row, every frame-boundary row
+    pair, the tail block, plus uniform random rows -- sorted, unique."""
+    rng = np.random.default_rng(seed)
+    fixed = [0, n - 1]
+    for fb in range(s, n, s):
+        fixed += [fb - 1, fb]
+    tail0 = (n // B) * B
+    fixed += list(range(tail0, n))
+    fixed = np.unique(np.clip(np.asarray(fixed, dtype=np.int64), 0, n - 1))
+    if fixed.size >= count:
+        pick = rng.choice(fixed, size=count, replace=False)
+        return np.sort(pick)
+    extra = rng.choice(n, size=min(n, count * 2), replace=False)
+    extra = np.setdiff1d(extra, fixed)[: count - fixed.size]
+    return np.sort(np.concatenate([fixed, extra]))
