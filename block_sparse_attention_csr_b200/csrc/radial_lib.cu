@@ -1,0 +1,443 @@
+// C ABI of the Radial Attention hot path (declared in include/radial.h).
+//
+// All device code of the library lives in this one translation unit (the
+// kernels are included from the .cuh files beside it), so the shared device
+// error word has a single definition.  Host code here only validates,
+// allocates the mask's arrays, encodes TMA descriptors and launches.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <string>
+
+#include "../../include/radial.h"
+#include "attn_bwd.cuh"
+#include "attn_fwd.cuh"
+#include "mask_build.cuh"
+#include "sm100_primitives.cuh"
+
+using namespace radial;
+
+// ---------------------------------------------------------------------------
+// errors and instrumentation
+// ---------------------------------------------------------------------------
+namespace {
+
+thread_local std::string t_last_error;
+std::atomic<int64_t> g_launches{0};
+
+radial_status fail(radial_status s, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  t_last_error = buf;
+  return s;
+}
+
+#define RADIAL_CUDA(call)                                                                        \
+  do {                                                                                           \
+    cudaError_t e_ = (call);                                                                     \
+    if (e_ != cudaSuccess) {                                                                     \
+      return fail(e_ == cudaErrorMemoryAllocation ? RADIAL_ENOMEM : RADIAL_ECUDA, "%s: %s (%s:%d)", \
+                  #call, cudaGetErrorString(e_), __FILE__, __LINE__);                            \
+    }                                                                                            \
+  } while (0)
+
+#define RADIAL_LAUNCHED()                                                                         \
+  do {                                                                                            \
+    g_launches.fetch_add(1, std::memory_order_relaxed);                                           \
+    cudaError_t e_ = cudaGetLastError();                                                          \
+    if (e_ != cudaSuccess)                                                                        \
+      return fail(RADIAL_ECUDA, "kernel launch: %s (%s:%d)", cudaGetErrorString(e_), __FILE__, __LINE__); \
+  } while (0)
+
+inline cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int sm_count() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) return 148;
+  return n;
+}
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no -lcuda).
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    cudaDriverEntryPointQueryResult q;
+    void* p = nullptr;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// 4D map over a bf16 [B, H, N, D] tensor (D contiguous), 128-row x 64-column
+// boxes with the 128-byte swizzle; rows past N read as zeros.
+radial_status make_bhnd_map(CUtensorMap* map, const void* base, const radial_desc& d) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return fail(RADIAL_ECUDA, "cuTensorMapEncodeTiled unavailable");
+  cuuint64_t dims[4] = {static_cast<cuuint64_t>(d.head_dim), static_cast<cuuint64_t>(d.n_tokens),
+                        static_cast<cuuint64_t>(d.heads), static_cast<cuuint64_t>(d.batch)};
+  cuuint64_t strides[3] = {static_cast<cuuint64_t>(d.stride_n) * 2, static_cast<cuuint64_t>(d.stride_h) * 2,
+                           static_cast<cuuint64_t>(d.stride_b) * 2};
+  cuuint32_t box[4] = {64, 128, 1, 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box,
+                  estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(RADIAL_ECUDA, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
+  return RADIAL_OK;
+}
+
+}  // namespace
+
+// ---------------------------------------------------------------------------
+// The mask object
+// ---------------------------------------------------------------------------
+struct TileLists {
+  int32_t nb = 0;
+  int64_t nnz = 0, n_full = 0;
+  int32_t *row_ptr = nullptr, *col_idx = nullptr, *col_ptr = nullptr, *row_idx = nullptr;
+  int32_t *row_order = nullptr, *col_order = nullptr;
+  uint8_t *kind = nullptr, *kind_t = nullptr;
+  void release() {
+    cudaFree(row_ptr); cudaFree(col_idx); cudaFree(col_ptr); cudaFree(row_idx);
+    cudaFree(row_order); cudaFree(col_order); cudaFree(kind); cudaFree(kind_t);
+    *this = TileLists();
+  }
+};
+
+struct radial_csr {
+  int32_t f = 0, s = 0, n = 0, B = 0, sink = 0, dense = 0, device = 0;
+  TileLists user;   // at the caller's block size
+  TileLists plan;   // at the kernels' 128-token tile (aliases `user` when B == 128)
+  bool plan_owned = false;
+};
+
+namespace {
+
+// From an nb x nb state matrix on the device, build CSR, CSC and orders.
+radial_status lists_from_states(const uint8_t* states, int32_t nb, TileLists& L, cudaStream_t st) {
+  L.nb = nb;
+  int32_t *row_cnt = nullptr, *col_cnt = nullptr;
+  unsigned long long* nfull = nullptr;
+  RADIAL_CUDA(cudaMalloc(&row_cnt, sizeof(int32_t) * nb));
+  RADIAL_CUDA(cudaMalloc(&col_cnt, sizeof(int32_t) * nb));
+  RADIAL_CUDA(cudaMalloc(&nfull, sizeof(unsigned long long)));
+  RADIAL_CUDA(cudaMalloc(&L.row_ptr, sizeof(int32_t) * (nb + 1)));
+  RADIAL_CUDA(cudaMalloc(&L.col_ptr, sizeof(int32_t) * (nb + 1)));
+  RADIAL_CUDA(cudaMalloc(&L.row_order, sizeof(int32_t) * nb));
+  RADIAL_CUDA(cudaMalloc(&L.col_order, sizeof(int32_t) * nb));
+  RADIAL_CUDA(cudaMemsetAsync(col_cnt, 0, sizeof(int32_t) * nb, st));
+  RADIAL_CUDA(cudaMemsetAsync(nfull, 0, sizeof(unsigned long long), st));
+  count_tiles_kernel<<<nb, 256, 0, st>>>(states, nb, row_cnt, col_cnt, nfull);
+  RADIAL_LAUNCHED();
+  exclusive_scan_kernel<<<1, 1024, 0, st>>>(row_cnt, nb, L.row_ptr);
+  RADIAL_LAUNCHED();
+  exclusive_scan_kernel<<<1, 1024, 0, st>>>(col_cnt, nb, L.col_ptr);
+  RADIAL_LAUNCHED();
+  int32_t nnz32 = 0;
+  unsigned long long nf = 0;
+  RADIAL_CUDA(cudaMemcpyAsync(&nnz32, L.row_ptr + nb, sizeof(int32_t), cudaMemcpyDeviceToHost, st));
+  RADIAL_CUDA(cudaMemcpyAsync(&nf, nfull, sizeof(nf), cudaMemcpyDeviceToHost, st));
+  RADIAL_CUDA(cudaStreamSynchronize(st));
+  L.nnz = nnz32;
+  L.n_full = static_cast<int64_t>(nf);
+  const size_t m = static_cast<size_t>(nnz32 > 0 ? nnz32 : 1);
+  RADIAL_CUDA(cudaMalloc(&L.col_idx, sizeof(int32_t) * m));
+  RADIAL_CUDA(cudaMalloc(&L.row_idx, sizeof(int32_t) * m));
+  RADIAL_CUDA(cudaMalloc(&L.kind, m));
+  RADIAL_CUDA(cudaMalloc(&L.kind_t, m));
+  compact_kernel<<<nb, 128, 0, st>>>(states, nb, false, L.row_ptr, L.col_idx, L.kind);
+  RADIAL_LAUNCHED();
+  compact_kernel<<<nb, 128, 0, st>>>(states, nb, true, L.col_ptr, L.row_idx, L.kind_t);
+  RADIAL_LAUNCHED();
+  const int rt = 256;
+  rank_by_count_kernel<<<(nb + rt - 1) / rt, rt, rt * sizeof(int32_t), st>>>(L.row_ptr, nb, L.row_order);
+  RADIAL_LAUNCHED();
+  rank_by_count_kernel<<<(nb + rt - 1) / rt, rt, rt * sizeof(int32_t), st>>>(L.col_ptr, nb, L.col_order);
+  RADIAL_LAUNCHED();
+  RADIAL_CUDA(cudaStreamSynchronize(st));
+  cudaFree(row_cnt);
+  cudaFree(col_cnt);
+  cudaFree(nfull);
+  return RADIAL_OK;
+}
+
+radial_status build_mask(int32_t f, int32_t s, int32_t B, int32_t sink, int32_t dense,
+                         radial_csr** out, cudaStream_t st) {
+  const int64_t n64 = static_cast<int64_t>(f) * s;
+  if (n64 > (1LL << 30)) return fail(RADIAL_EINVAL, "frames * tokens_per_frame = %lld exceeds 2^30", (long long)n64);
+  const int32_t n = static_cast<int32_t>(n64);
+  const int32_t nb = (n + B - 1) / B;
+  if (nb > 32768) return fail(RADIAL_EUNSUPPORTED, "%d blocks per side exceeds 32768", nb);
+  radial_csr* c = new (std::nothrow) radial_csr();
+  if (!c) return fail(RADIAL_ENOMEM, "host allocation failed");
+  c->f = f; c->s = s; c->n = n; c->B = B; c->sink = sink; c->dense = dense;
+  cudaGetDevice(&c->device);
+  uint8_t* states = nullptr;
+  uint8_t* states128 = nullptr;
+  radial_status rs = RADIAL_OK;
+  auto cleanup = [&](radial_status r) {
+    cudaStreamSynchronize(st);
+    cudaFree(states);
+    cudaFree(states128);
+    if (r != RADIAL_OK) {
+      if (c->plan_owned) c->plan.release();
+      c->user.release();
+      delete c;
+    }
+    return r;
+  };
+  if (cudaMalloc(&states, static_cast<size_t>(nb) * nb) != cudaSuccess)
+    return cleanup(fail(RADIAL_ENOMEM, "cannot allocate %d x %d tile states", nb, nb));
+  MaskGeom g{f, s, n, B, nb, sink};
+  dim3 grid((nb + 127) / 128, nb);
+  classify_tiles_kernel<<<grid, 128, 0, st>>>(g, states);
+  g_launches.fetch_add(1);
+  if (cudaGetLastError() != cudaSuccess) return cleanup(fail(RADIAL_ECUDA, "classify_tiles launch failed"));
+  rs = lists_from_states(states, nb, c->user, st);
+  if (rs != RADIAL_OK) return cleanup(rs);
+  if (B == 128) {
+    c->plan = c->user;
+    c->plan_owned = false;
+  } else {
+    const int32_t nt = (n + 127) / 128;
+    if (cudaMalloc(&states128, static_cast<size_t>(nt) * nt) != cudaSuccess)
+      return cleanup(fail(RADIAL_ENOMEM, "cannot allocate %d x %d tile plan", nt, nt));
+    dim3 g2((nt + 127) / 128, nt);
+    coarsen_states_kernel<<<g2, 128, 0, st>>>(states, nb, states128, nt);
+    g_launches.fetch_add(1);
+    if (cudaGetLastError() != cudaSuccess) return cleanup(fail(RADIAL_ECUDA, "coarsen launch failed"));
+    c->plan_owned = true;
+    rs = lists_from_states(states128, nt, c->plan, st);
+    if (rs != RADIAL_OK) return cleanup(rs);
+  }
+  *out = c;
+  return cleanup(RADIAL_OK);
+}
+
+}  // namespace
+
+// ---------------------------------------------------------------------------
+// ABI
+// ---------------------------------------------------------------------------
+extern "C" {
+
+void radial_params_default(radial_params* p) {
+  if (!p) return;
+  std::memset(p, 0, sizeof(*p));
+  p->sink = 1;
+  p->central_band = 1;
+  p->width_scale = 2;
+}
+
+radial_status radial_mask_build(int32_t frames, int32_t tokens_per_frame, int32_t block,
+                                const radial_params* params, radial_csr** out, void* stream) {
+  if (!out) return fail(RADIAL_EINVAL, "out is NULL");
+  *out = nullptr;
+  radial_params def;
+  radial_params_default(&def);
+  const radial_params* pr = params ? params : &def;
+  for (int i = 0; i < 5; ++i)
+    if (pr->reserved[i] != 0) return fail(RADIAL_EINVAL, "params.reserved[%d] must be 0", i);
+  if (pr->sink != 0 && pr->sink != 1) return fail(RADIAL_EINVAL, "params.sink must be 0 or 1");
+  if (pr->central_band != 1) return fail(RADIAL_EUNSUPPORTED, "only central_band = 1 is implemented");
+  if (pr->width_scale != 2) return fail(RADIAL_EUNSUPPORTED, "only width_scale = 2 is implemented");
+  if (frames < 1 || tokens_per_frame < 1) return fail(RADIAL_EINVAL, "frames and tokens_per_frame must be >= 1");
+  if (block != 64 && block != 128) return fail(RADIAL_EUNSUPPORTED, "block must be 64 or 128");
+  return build_mask(frames, tokens_per_frame, block, pr->sink, 0, out, as_stream(stream));
+}
+
+radial_status radial_mask_build_dense(int32_t n_tokens, int32_t block, radial_csr** out, void* stream) {
+  if (!out) return fail(RADIAL_EINVAL, "out is NULL");
+  *out = nullptr;
+  if (n_tokens < 1) return fail(RADIAL_EINVAL, "n_tokens must be >= 1");
+  if (block != 64 && block != 128) return fail(RADIAL_EUNSUPPORTED, "block must be 64 or 128");
+  // One frame of n tokens: distance 0 everywhere, so every pair is allowed.
+  return build_mask(1, n_tokens, block, 0, 1, out, as_stream(stream));
+}
+
+radial_status radial_csr_info(const radial_csr* c, radial_csr_info_t* info) {
+  if (!c || !info) return fail(RADIAL_EINVAL, "NULL argument");
+  std::memset(info, 0, sizeof(*info));
+  info->frames = c->f;
+  info->tokens_per_frame = c->s;
+  info->n_tokens = c->n;
+  info->block = c->B;
+  info->n_blocks = c->user.nb;
+  info->sink = c->sink;
+  info->dense = c->dense;
+  info->nnz = c->user.nnz;
+  info->n_full = c->user.n_full;
+  return RADIAL_OK;
+}
+
+radial_status radial_csr_copy_to_host(const radial_csr* c, int32_t* row_ptr, int32_t* col_idx,
+                                      uint8_t* kind, int32_t* col_ptr, int32_t* row_idx,
+                                      uint8_t* kind_t, int32_t* row_order, int32_t* col_order) {
+  if (!c) return fail(RADIAL_EINVAL, "csr is NULL");
+  const TileLists& L = c->user;
+  const size_t nb = static_cast<size_t>(L.nb), nnz = static_cast<size_t>(L.nnz);
+  if (row_ptr) RADIAL_CUDA(cudaMemcpy(row_ptr, L.row_ptr, 4 * (nb + 1), cudaMemcpyDeviceToHost));
+  if (col_ptr) RADIAL_CUDA(cudaMemcpy(col_ptr, L.col_ptr, 4 * (nb + 1), cudaMemcpyDeviceToHost));
+  if (col_idx) RADIAL_CUDA(cudaMemcpy(col_idx, L.col_idx, 4 * nnz, cudaMemcpyDeviceToHost));
+  if (row_idx) RADIAL_CUDA(cudaMemcpy(row_idx, L.row_idx, 4 * nnz, cudaMemcpyDeviceToHost));
+  if (kind) RADIAL_CUDA(cudaMemcpy(kind, L.kind, nnz, cudaMemcpyDeviceToHost));
+  if (kind_t) RADIAL_CUDA(cudaMemcpy(kind_t, L.kind_t, nnz, cudaMemcpyDeviceToHost));
+  if (row_order) RADIAL_CUDA(cudaMemcpy(row_order, L.row_order, 4 * nb, cudaMemcpyDeviceToHost));
+  if (col_order) RADIAL_CUDA(cudaMemcpy(col_order, L.col_order, 4 * nb, cudaMemcpyDeviceToHost));
+  return RADIAL_OK;
+}
+
+void radial_csr_free(radial_csr* c) {
+  if (!c) return;
+  cudaDeviceSynchronize();
+  if (c->plan_owned) c->plan.release();
+  c->user.release();
+  delete c;
+}
+
+}  // extern "C"
+
+// ---------------------------------------------------------------------------
+// attention validation shared by forward and backward
+// ---------------------------------------------------------------------------
+namespace {
+
+radial_status check_desc(const radial_csr* c, const radial_desc* d) {
+  if (!c || !d) return fail(RADIAL_EINVAL, "NULL csr or desc");
+  if (d->batch < 1 || d->heads < 1) return fail(RADIAL_EINVAL, "batch and heads must be >= 1");
+  if (d->n_tokens != c->n) return fail(RADIAL_EINVAL, "desc.n_tokens %d != mask n %d", d->n_tokens, c->n);
+  if (d->head_dim != 64 && d->head_dim != 128) return fail(RADIAL_EUNSUPPORTED, "head_dim must be 64 or 128");
+  if (d->reserved != 0) return fail(RADIAL_EINVAL, "desc.reserved must be 0");
+  if (d->stride_n < d->head_dim || d->stride_h < 1 || d->stride_b < 1)
+    return fail(RADIAL_EINVAL, "strides must cover head_dim");
+  if ((d->stride_n * 2) % 16 || (d->stride_h * 2) % 16 || (d->stride_b * 2) % 16)
+    return fail(RADIAL_EINVAL, "strides * 2 bytes must be multiples of 16");
+  if (static_cast<int64_t>(d->batch) * d->heads * ((d->n_tokens + 127) / 128) > 0x7fffffffLL)
+    return fail(RADIAL_EUNSUPPORTED, "too many work items");
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev != c->device) return fail(RADIAL_EINVAL, "mask built on device %d, current device %d", c->device, dev);
+  return RADIAL_OK;
+}
+
+float softmax_scale(const radial_desc* d) {
+  return d->scale > 0.f ? d->scale : 1.0f / std::sqrt(static_cast<float>(d->head_dim));
+}
+
+template <int D>
+radial_status launch_fwd(const radial_csr* c, const radial_desc* d, const void* q, const void* k,
+                         const void* v, void* o, float* lse, cudaStream_t st) {
+  CUtensorMap mq, mk, mv;
+  radial_status rs;
+  if ((rs = make_bhnd_map(&mq, q, *d)) != RADIAL_OK) return rs;
+  if ((rs = make_bhnd_map(&mk, k, *d)) != RADIAL_OK) return rs;
+  if ((rs = make_bhnd_map(&mv, v, *d)) != RADIAL_OK) return rs;
+  FwdParams p;
+  p.row_ptr = c->plan.row_ptr;
+  p.col_idx = c->plan.col_idx;
+  p.kind = c->plan.kind;
+  p.order = c->plan.row_order;
+  p.nt = c->plan.nb;
+  p.f = c->f;
+  p.s = c->s;
+  p.n = c->n;
+  p.sink = c->sink;
+  p.heads = d->heads;
+  p.items = d->batch * d->heads * c->plan.nb;
+  p.o_sb = d->stride_b;
+  p.o_sh = d->stride_h;
+  p.o_sn = d->stride_n;
+  p.o = reinterpret_cast<__nv_bfloat16*>(o);
+  p.lse = lse;
+  p.scale_log2 = softmax_scale(d) * 1.4426950408889634f;
+  const int smem = FwdCfg<D>::SMEM_BYTES;
+  RADIAL_CUDA(cudaFuncSetAttribute(radial_fwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
+  const int grid = p.items < sm_count() ? p.items : sm_count();
+  radial_fwd_kernel<D><<<grid, 192, smem, st>>>(mq, mk, mv, p);
+  RADIAL_LAUNCHED();
+  return RADIAL_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+radial_status radial_attn_fwd(const radial_csr* c, const radial_desc* d, const void* q, const void* k,
+                              const void* v, void* o, float* lse, void* stream) {
+  radial_status rs = check_desc(c, d);
+  if (rs != RADIAL_OK) return rs;
+  if (!q || !k || !v || !o || !lse) return fail(RADIAL_EINVAL, "NULL tensor pointer");
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
+    return fail(RADIAL_EINVAL, "tensor pointers must be 16-byte aligned");
+  if (d->head_dim == 128) return launch_fwd<128>(c, d, q, k, v, o, lse, as_stream(stream));
+  return launch_fwd<64>(c, d, q, k, v, o, lse, as_stream(stream));
+}
+
+size_t radial_attn_bwd_workspace_size(const radial_desc* d) {
+  if (!d || d->batch < 1 || d->heads < 1 || d->n_tokens < 1 || d->head_dim < 1) return 0;
+  const size_t rows = static_cast<size_t>(d->batch) * d->heads * d->n_tokens;
+  const size_t dq = rows * d->head_dim * sizeof(float);
+  const size_t dr = rows * sizeof(float);
+  return ((dq + 255) & ~size_t(255)) + ((dr + 255) & ~size_t(255));
+}
+
+radial_status radial_attn_bwd(const radial_csr* c, const radial_desc* d, const void* dout, const void* q,
+                              const void* k, const void* v, const void* o, const float* lse, void* dq,
+                              void* dk, void* dv, void* workspace, size_t workspace_bytes, void* stream) {
+  radial_status rs = check_desc(c, d);
+  if (rs != RADIAL_OK) return rs;
+  (void)dout; (void)q; (void)k; (void)v; (void)o; (void)lse; (void)dq; (void)dk; (void)dv;
+  (void)workspace; (void)workspace_bytes; (void)stream;
+  return fail(RADIAL_EUNSUPPORTED, "backward not built yet");
+}
+
+radial_status radial_device_status(void* stream) {
+  RADIAL_CUDA(cudaStreamSynchronize(as_stream(stream)));
+  int flag = 0;
+  RADIAL_CUDA(cudaMemcpyFromSymbol(&flag, g_device_error, sizeof(int)));
+  if (flag != 0) {
+    const int zero = 0;
+    RADIAL_CUDA(cudaMemcpyToSymbol(g_device_error, &zero, sizeof(int)));
+    return fail(RADIAL_EDEVICE, "a kernel aborted after a bounded wait ran out (code %d)", flag);
+  }
+  RADIAL_CUDA(cudaGetLastError());
+  return RADIAL_OK;
+}
+
+const char* radial_status_str(radial_status s) {
+  switch (s) {
+    case RADIAL_OK: return "ok";
+    case RADIAL_EINVAL: return "invalid argument";
+    case RADIAL_EUNSUPPORTED: return "unsupported";
+    case RADIAL_ENOMEM: return "out of memory";
+    case RADIAL_ECUDA: return "CUDA error";
+    case RADIAL_EDEVICE: return "device-side abort";
+  }
+  return "unknown status";
+}
+
+const char* radial_last_error(void) { return t_last_error.c_str(); }
+
+int64_t radial_launch_count(void) { return g_launches.load(); }
+
+}  // extern "C"

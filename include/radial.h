@@ -1,0 +1,185 @@
+/*
+ * radial.h -- C ABI of the B200 (sm_100a) Radial Attention hot path.
+ *
+ * The operation: masked softmax attention O = softmax(Q K^T * scale + M) V
+ * (the sparse-attention equation, Eq.2, of "Paper review: Radial Attention:
+ * O(n log n) Sparse Attention with Energy Decay for Long Video Generation",
+ * jaehun.me, §3), where M is the static spatiotemporal radial mask of that
+ * page's §4.2 (temporal bands, Fig.5a; shrinking spatial diagonal, Fig.5b;
+ * the 4D mask Eq.4 flattened to 2D; the attention sink of App. A.1 Eq.8),
+ * executed block-sparsely over the active tiles of a block CSR (§4.2: the
+ * implementation computes in 128x128 token blocks).  The backward pass is
+ * the one the LoRA length-extension fine-tuning of §4.3 needs.
+ *
+ * Mask reading (the printed formulas were lost; the plain reading, which
+ * reproduces the page's worked toy example exactly): tokens a = i*s + k
+ * (frame i, row-major position k), b = j*s + l, d = |i - j|,
+ * r = floor(log2(max(d,1))), h = floor(s / 2^r) - 1, c = ceil(2^r / s);
+ * (a, b) is allowed iff (sink and j == 0) or (h >= 0 and |k - l| <= h) or
+ * (h < 0 and d mod c == 0 and k == l).
+ *
+ * Conventions shared by every call
+ *  - Every call is asynchronous on `stream` (a cudaStream_t passed as void*;
+ *    NULL = the legacy default stream) unless its comment says otherwise.
+ *  - All arguments are validated on the host before anything is launched; a
+ *    call that returns an error has launched nothing.
+ *  - No exception crosses the ABI.  CUDA failures map to RADIAL_ECUDA; the
+ *    text of the last error on the calling thread is radial_last_error().
+ *  - Kernels never wait without bound: a producer/consumer wait that exceeds
+ *    its limit (about 2 s) aborts the kernel and records RADIAL_EDEVICE,
+ *    which radial_device_status() reports (and clears).
+ *  - The caller owns every tensor and workspace buffer; the library owns a
+ *    radial_csr from its build call until radial_csr_free().
+ */
+#ifndef RADIAL_H_
+#define RADIAL_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum radial_status {
+  RADIAL_OK = 0,
+  RADIAL_EINVAL = 1,        /* invalid argument: null, misaligned, inconsistent sizes */
+  RADIAL_EUNSUPPORTED = 2,  /* well-formed but outside what the kernels implement */
+  RADIAL_ENOMEM = 3,        /* a device or host allocation failed */
+  RADIAL_ECUDA = 4,         /* a CUDA runtime or driver call failed */
+  RADIAL_EDEVICE = 5        /* a kernel aborted after a bounded wait ran out */
+} radial_status;
+
+/* Mask parameters.  sink: 1 = every query also attends to all tokens of frame
+ * 0 (App. A.1 Eq.8; default 1).  central_band: frame distances <= this are
+ * dense (the authors' "width of central band" ablation; only the default 1 is
+ * implemented).  width_scale: width ratio between consecutive temporal bands
+ * (their "width scale" ablation; only the default 2 is implemented).
+ * reserved: must be zero. */
+typedef struct radial_params {
+  int32_t sink;
+  int32_t central_band;
+  int32_t width_scale;
+  int32_t reserved[5];
+} radial_params;
+
+/* Fill *p with the defaults {sink = 1, central_band = 1, width_scale = 2}. */
+void radial_params_default(radial_params* p);
+
+/* Opaque block-sparse mask: the block CSR and CSC of active tiles plus the
+ * kernels' schedules, all in device memory owned by the library. */
+typedef struct radial_csr radial_csr;
+
+typedef struct radial_csr_info_t {
+  int32_t frames;            /* f */
+  int32_t tokens_per_frame;  /* s */
+  int32_t n_tokens;          /* n = f * s */
+  int32_t block;             /* B: tile edge in tokens */
+  int32_t n_blocks;          /* ceil(n / B): q-blocks = k-blocks */
+  int32_t sink;
+  int32_t dense;             /* 1 if built by radial_mask_build_dense */
+  int32_t reserved;
+  int64_t nnz;               /* active tiles */
+  int64_t n_full;            /* active tiles with every pair allowed */
+  int64_t allowed_pairs;     /* reserved: 0 (not computed by the builder) */
+} radial_csr_info_t;
+
+/* Build the block CSR of the radial mask for f frames of s tokens with square
+ * B x B tiles (§4.2: block-wise execution).  A tile (qb, kb) is ACTIVE iff it
+ * holds at least one allowed pair of tokens < n; FULL (kind 1) iff both
+ * blocks lie inside [0, n) and every pair in it is allowed; else PARTIAL
+ * (kind 2).  Columns of a row are ascending; the CSC lists, per key block,
+ * its active query blocks ascending; row_order / col_order list blocks by
+ * active-tile count descending, ties by index ascending.
+ * Runs on the device on `stream` and SYNCHRONISES it (the tile count sizes the
+ * allocation).  Constraints: f >= 1, s >= 1, f*s < 2^31, B in {64, 128},
+ * ceil(n/B) <= 32768.  On success *out owns device memory until
+ * radial_csr_free.  Errors: RADIAL_EINVAL (bad sizes, null out/params,
+ * non-zero reserved), RADIAL_EUNSUPPORTED (non-default central_band or
+ * width_scale, other B), RADIAL_ENOMEM, RADIAL_ECUDA. */
+radial_status radial_mask_build(int32_t frames, int32_t tokens_per_frame, int32_t block,
+                                const radial_params* params, radial_csr** out, void* stream);
+
+/* The all-ones mask of n tokens (dense attention, Eq.1 of the same page, run
+ * through the same kernels): every tile active, FULL except tail tiles.  It
+ * is the dense comparator and the dense-layer / dense-warm-up mode the
+ * authors use in their first layers and steps.  Same contract as
+ * radial_mask_build. */
+radial_status radial_mask_build_dense(int32_t n_tokens, int32_t block, radial_csr** out,
+                                      void* stream);
+
+/* Sizes of a built mask.  Host only; no device work. */
+radial_status radial_csr_info(const radial_csr* csr, radial_csr_info_t* info);
+
+/* Copy the mask to host arrays (each may be NULL to skip it).  Sizes:
+ * row_ptr, col_ptr: n_blocks + 1 int32; col_idx, row_idx: nnz int32;
+ * kind, kind_t: nnz uint8 (1 FULL, 2 PARTIAL; kind_t in CSC order);
+ * row_order, col_order: n_blocks int32.  Synchronous (blocks the host). */
+radial_status radial_csr_copy_to_host(const radial_csr* csr, int32_t* row_ptr, int32_t* col_idx,
+                                      uint8_t* kind, int32_t* col_ptr, int32_t* row_idx,
+                                      uint8_t* kind_t, int32_t* row_order, int32_t* col_order);
+
+/* Release a mask (waits for the device to be done with it).  NULL is a no-op. */
+void radial_csr_free(radial_csr* csr);
+
+/* Shape and layout of the attention tensors.  Q, K, V, O, dO, dQ, dK, dV are
+ * bf16 [batch, heads, n_tokens, head_dim] with head_dim contiguous and the
+ * element strides given here (shared by all eight tensors); every base
+ * pointer and stride * 2 bytes must be 16-byte aligned.  LSE is fp32
+ * [batch, heads, n_tokens], contiguous.  head_dim in {64, 128}.
+ * scale: softmax scale; <= 0 selects 1/sqrt(head_dim) (Eq.1's scaling). */
+typedef struct radial_desc {
+  int32_t batch;
+  int32_t heads;
+  int32_t n_tokens;
+  int32_t head_dim;
+  int64_t stride_b;
+  int64_t stride_h;
+  int64_t stride_n;
+  float scale;
+  int32_t reserved;
+} radial_desc;
+
+/* Forward (Eq.2 under the mask): writes O (bf16, rows normalised) and
+ * LSE = ln(sum_b exp(scale * q.k_b)) over allowed keys (fp32, natural log) for
+ * every (batch, head, token).  The same mask serves every batch entry and
+ * head (it depends on positions only, §4.2).  desc->n_tokens must equal the
+ * mask's n.  Reads q, k, v; writes o, lse; no workspace; asynchronous. */
+radial_status radial_attn_fwd(const radial_csr* csr, const radial_desc* desc, const void* q,
+                              const void* k, const void* v, void* o, float* lse, void* stream);
+
+/* Bytes of device workspace radial_attn_bwd needs for this shape (fp32 dQ
+ * accumulator plus per-row dO.O sums).  Host only. */
+size_t radial_attn_bwd_workspace_size(const radial_desc* desc);
+
+/* Backward of Eq.2 under the mask (the gradients LoRA fine-tuning, §4.3,
+ * back-propagates through attention): given dO, the forward's inputs, its O
+ * and LSE, writes dQ, dK, dV (bf16, same layout).  `workspace` is caller-owned
+ * device memory of at least radial_attn_bwd_workspace_size(desc) bytes,
+ * 256-byte aligned; its contents on entry do not matter and on exit are
+ * unspecified.  Asynchronous. */
+radial_status radial_attn_bwd(const radial_csr* csr, const radial_desc* desc, const void* dout,
+                              const void* q, const void* k, const void* v, const void* o,
+                              const float* lse, void* dq, void* dk, void* dv, void* workspace,
+                              size_t workspace_bytes, void* stream);
+
+/* Synchronise `stream` and report whether any kernel of this library aborted
+ * on a bounded wait since the last call (RADIAL_EDEVICE, then cleared), or a
+ * CUDA error is pending (RADIAL_ECUDA).  RADIAL_OK otherwise. */
+radial_status radial_device_status(void* stream);
+
+/* Static text for a status code. */
+const char* radial_status_str(radial_status s);
+
+/* Text of the last error raised on the calling thread ("" if none). */
+const char* radial_last_error(void);
+
+/* Number of kernel launches this library has issued in this process (all
+ * threads, all devices).  Host counter, for instrumentation. */
+int64_t radial_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* RADIAL_H_ */

@@ -1,0 +1,146 @@
+"""Forward parity: the CUDA path (through the C ABI) against the fp64 CPU
+reference on the same seeded bf16 inputs.
+
+Tolerances (from the acceptance criteria of the workload definitions):
+O max-abs <= 2e-2 and mean-abs <= 2e-3 against fp64; LSE max-abs <= 1e-3
+(fp32 accumulation of at most 5e5 terms on logits of magnitude < 10: relative
+error ~1e-6, so 1e-3 leaves three orders of margin while still catching a
+wrong scale, base or mask).
+"""
+
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import block_sparse_attention_csr_b200 as rb
+from block_sparse_attention_csr_b200 import inputs as I
+from oracle import attention as A
+from tests import oracle_pool
+
+pytestmark = pytest.mark.gpu
+
+O_MAX, O_MEAN, LSE_MAX = 2e-2, 2e-3, 1e-3
+DEV = "cuda"
+
+
+def _run_gpu(q, k, v, f, s, block, sink, dense=False):
+    csr = rb.radial_mask_build_dense(f * s, block) if dense else rb.radial_mask_build(f, s, block, sink=sink)
+    o, lse = rb.radial_attn_fwd(csr, q, k, v)
+    rb.radial_device_status()
+    return o, lse
+
+
+def _check(o_gpu, lse_gpu, o_ref, lse_ref, what):
+    err = np.abs(o_gpu.astype(np.float64) - o_ref)
+    lerr = np.abs(lse_gpu.astype(np.float64) - lse_ref)
+    assert np.isfinite(o_gpu).all(), what
+    assert err.max() <= O_MAX, f"{what}: O max-abs {err.max():.3e}"
+    assert err.mean() <= O_MEAN, f"{what}: O mean-abs {err.mean():.3e}"
+    assert lerr.max() <= LSE_MAX, f"{what}: LSE max-abs {lerr.max():.3e}"
+
+
+def _full_check(q, k, v, f, s, block, sink, dense=False, what=""):
+    o, lse = _run_gpu(q, k, v, f, s, block, sink, dense)
+    ff, ss = (1, f * s) if dense else (f, s)
+    o_ref, l_ref = A.radial_forward(q.float().cpu().numpy(), k.float().cpu().numpy(),
+                                    v.float().cpu().numpy(), ff, ss, bool(sink) and not dense)
+    _check(o.float().cpu().numpy(), lse.cpu().numpy(), o_ref, l_ref, what)
+
+
+def test_tiny_config_all_rows():
+    wl = I.WORKLOADS["tiny"]
+    q32, k32, v32 = I.draw_fp32(wl, backward=False)
+    q, k, v = (x.to(torch.bfloat16).to(DEV) for x in (q32, k32, v32))
+    _full_check(q, k, v, wl.frames, wl.tokens_per_frame, wl.block, 1, what="tiny")
+
+
+SMALL = [
+    # batch, heads, head_dim, frames, tokens_per_frame, block, sink, seed
+    (1, 2, 128, 5, 200, 128, 1, 11),     # ragged tail (1000 = 7*128 + 104)
+    (2, 2, 64, 7, 300, 64, 0, 12),       # batch > 1, block 64, sink off
+    (1, 1, 128, 32, 256, 64, 1, 13),     # many tiles, block 64 / d 128
+    (1, 1, 64, 40, 3, 128, 1, 14),       # s < block: one tile spans many frames
+    (1, 1, 128, 64, 4, 64, 0, 15),       # sampled-diagonal branch (width < 1)
+    (1, 3, 128, 2, 700, 128, 0, 16),     # f <= 2: the mask is all-ones
+    (1, 1, 64, 1, 1, 64, 1, 17),         # a single token
+    (1, 2, 128, 9, 1000, 128, 1, 18),    # frames not aligned to tiles
+    (1, 1, 128, 12, 1560, 128, 1, 19),   # Wan-like frame size, 12 frames
+]
+
+
+@pytest.mark.parametrize("Bn,H,D,f,s,block,sink,seed", SMALL)
+def test_small_all_rows(Bn, H, D, f, s, block, sink, seed):
+    wl = I.small_workload("t", Bn, H, D, f, s, block, seed)
+    q, k, v = I.draw(wl, device=DEV, backward=False)
+    _full_check(q, k, v, f, s, block, sink, what=f"{(Bn, H, D, f, s, block, sink)}")
+
+
+def test_dense_mask_equals_dense_attention():
+    wl = I.small_workload("d", 1, 2, 128, 1, 1500, 128, 21)
+    q, k, v = I.draw(wl, device=DEV, backward=False)
+    _full_check(q, k, v, 1, 1500, 128, 0, dense=True, what="dense")
+
+
+def test_strided_layout():
+    """[B, N, H, D] storage viewed as [B, H, N, D] (non-contiguous heads)."""
+    g = torch.Generator(device="cpu").manual_seed(22)
+    Bn, H, N, D, f, s = 1, 3, 1200, 128, 6, 200
+    base = [torch.randn(Bn, N, H, D, generator=g).to(torch.bfloat16).to(DEV) for _ in range(3)]
+    q, k, v = (t.permute(0, 2, 1, 3) for t in base)
+    o = torch.empty(Bn, N, H, D, dtype=torch.bfloat16, device=DEV).permute(0, 2, 1, 3)
+    csr = rb.radial_mask_build(f, s, 128, sink=1)
+    o, lse = rb.radial_attn_fwd(csr, q, k, v, o=o)
+    rb.radial_device_status()
+    o_ref, l_ref = A.radial_forward(q.float().cpu().numpy(), k.float().cpu().numpy(),
+                                    v.float().cpu().numpy(), f, s, True)
+    _check(o.float().cpu().numpy(), lse.cpu().numpy(), o_ref, l_ref, "strided")
+
+
+def test_repeated_calls_are_deterministic():
+    wl = I.small_workload("r", 1, 4, 128, 9, 1000, 128, 23)
+    q, k, v = I.draw(wl, device=DEV, backward=False)
+    csr = rb.radial_mask_build(9, 1000, 128, sink=1)
+    o1, l1 = rb.radial_attn_fwd(csr, q, k, v)
+    o2, l2 = rb.radial_attn_fwd(csr, q, k, v)
+    rb.radial_device_status()
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)
+
+
+def _sampled_check(name, rows_per_head, heads=None):
+    wl = I.WORKLOADS[name]
+    q, k, v = I.draw(wl, device=DEV, backward=False)
+    csr = rb.radial_mask_build(wl.frames, wl.tokens_per_frame, wl.block, sink=1)
+    o, lse = rb.radial_attn_fwd(csr, q, k, v)
+    rb.radial_device_status()
+    n = wl.n
+    heads = range(wl.heads) if heads is None else heads
+    tasks, keep = [], []
+    scale = 1.0 / np.sqrt(wl.head_dim)
+    for h in heads:
+        rows = A.sample_rows(n, rows_per_head, wl.tokens_per_frame, wl.block, seed=1000 + h)
+        ridx = torch.as_tensor(rows, device=DEV)
+        tasks.append((q[0, h, ridx].float().cpu().numpy().astype(np.float64),
+                      k[0, h].float().cpu().numpy(), v[0, h].float().cpu().numpy(),
+                      rows, wl.frames, wl.tokens_per_frame, True, scale))
+        keep.append((o[0, h, ridx].float().cpu().numpy(), lse[0, h, ridx].cpu().numpy()))
+    res = oracle_pool.run("fwd_rows", tasks)
+    o_g = np.concatenate([a for a, _ in keep])
+    l_g = np.concatenate([b for _, b in keep])
+    o_r = np.concatenate([a for a, _ in res])
+    l_r = np.concatenate([b for _, b in res])
+    _check(o_g, l_g, o_r, l_r, name)
+
+
+def test_wan480p_sampled_rows():
+    _sampled_check("wan480p", 4096)
+
+
+def test_hunyuan720p_sampled_rows():
+    _sampled_check("hunyuan720p", 4096)
+
+
+@pytest.mark.slow
+def test_hunyuan720p_4x_sampled_rows():
+    _sampled_check("hunyuan720p_4x", int(os.environ.get("RADIAL_4X_ROWS", "4096")))
