@@ -1,0 +1,483 @@
+"""Benchmark of the radial block-sparse attention hot path on B200.
+
+Default workload: the HunyuanVideo-shaped 720p 5 s self-attention (batch 1,
+24 heads, head_dim 128, 33 frames x 3600 tokens = 118,800 tokens, 128x128
+tiles, attention sink on), forward call -- the shape the throughput target is
+stated on.  A step is one radial_attn_fwd call over the whole batch; the
+static mask is built once per shape (it depends on positions only) and its
+build time is reported beside the step.  With --workload hunyuan720p_4x a
+step is the 4x-length LoRA fine-tuning pass: forward plus backward.
+
+Prints one JSON line (rank 0).  Multi-GPU (torchrun): every rank runs the
+same workload on its own GPU (independent problems, no collective on the data
+path; weak scaling); the step time is the max over ranks.
+
+--impl reference times the CPU reference (oracle/) on the host cores instead.
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "ms and TFLOP/s (active tiles) per attention call, % of tensor peak, speedup vs dense"
+
+
+def _peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as fh:
+            pk = json.load(fh)
+        return float(pk["bf16_tflops"]), float(pk["bf16_tflops_sustained"]), float(pk["hbm_gbs"]), "measured"
+    except Exception:
+        return 1590.0, 1400.0, 6650.0, "fallback"
+
+
+def _cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+# ---------------------------------------------------------------------------
+# workload accounting (host-side integers only)
+# ---------------------------------------------------------------------------
+
+def tile_flops(wl, nnz, backward=False):
+    """Algorithmic flops on active tiles: 4*B^2*d per tile forward (QK^T and PV),
+    10*B^2*d backward (five tile GEMMs), times batch*heads."""
+    per = 4 if not backward else 10
+    return per * wl.block * wl.block * wl.head_dim * nnz * wl.batch * wl.heads
+
+
+def whole_job_tflops(flops_per_rank, world, ms_max):
+    """Whole-job throughput: every rank runs one replica of the workload
+    (independent problems), so the job does world * flops_per_rank in the
+    slowest rank's time."""
+    return world * flops_per_rank / (ms_max * 1e-3) / 1e12
+
+
+def max_over_ranks(ms, world, device=None):
+    """Step time as the max over ranks (all-reduce MAX; identity at world 1)."""
+    if world <= 1:
+        return float(ms)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(ms)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def config_of(wl, nnz):
+    return {"workload": wl.name, "batch": wl.batch, "heads": wl.heads, "head_dim": wl.head_dim,
+            "frames": wl.frames, "tokens_per_frame": wl.tokens_per_frame, "n_tokens": wl.n,
+            "block": wl.block, "sink": True, "active_tiles": int(nnz),
+            "l2": "inputs larger than L2 (no flush): Q,K,V %.2f GB per step" % (3 * wl.batch * wl.heads * wl.n * wl.head_dim * 2 / 1e9)}
+
+
+# ---------------------------------------------------------------------------
+# clocks sampled during the timed region
+# ---------------------------------------------------------------------------
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, phys_index):
+        self.idx = phys_index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "200",
+                 "-i", str(self.idx)], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        sm, mx, reasons, power = [], None, set(), []
+        for ln in self.lines:
+            p = [x.strip() for x in ln.split(",")]
+            if len(p) < 9:
+                continue
+            try:
+                sm.append(float(p[1]))
+                mx = float(p[2])
+                power.append(float(p[3]))
+            except ValueError:
+                continue
+            for name, val in zip(("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"), p[5:9]):
+                if val.lower().startswith("active"):
+                    reasons.add(name)
+        sm.sort()
+        med = sm[len(sm) // 2] if sm else None
+        return {"sm_mhz": med, "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm),
+                "power_w_max": max(power) if power else None}
+
+
+# ---------------------------------------------------------------------------
+# CPU reference timing (oracle) -- bounded sample
+# ---------------------------------------------------------------------------
+
+def oracle_rows_timing(wl, q_rows, k_head, v_head, rows, budget_s):
+    """Time the CPU reference on query rows of one head; returns (seconds, rows done)."""
+    from oracle import attention as A
+    import numpy as np
+    n = wl.n
+    q = np.zeros((n, wl.head_dim))
+    done, t0 = 0, time.perf_counter()
+    chunk = 256
+    while done < len(rows):
+        r = rows[done:done + chunk]
+        q[r] = q_rows[done:done + chunk]
+        A.forward_rows(q, k_head, v_head, r, wl.frames, wl.tokens_per_frame, True, chunk=chunk)
+        done += len(r)
+        if time.perf_counter() - t0 > budget_s:
+            break
+    return time.perf_counter() - t0, done
+
+
+def cpu_baseline(wl, nnz, q, k, v, budget_s=15.0, backward=False):
+    import numpy as np
+    from oracle import attention as A
+    rows = A.sample_rows(wl.n, 8192, wl.tokens_per_frame, wl.block, seed=77)
+    np.random.default_rng(5).shuffle(rows)
+    kh = k[0, 0].float().cpu().numpy().astype(np.float64)
+    vh = v[0, 0].float().cpu().numpy().astype(np.float64)
+    qr = q[0, 0].float().cpu().numpy()[rows].astype(np.float64)
+    secs, done = oracle_rows_timing(wl, qr, kh, vh, rows, budget_s)
+    total_rows = wl.batch * wl.heads * wl.n
+    full_s = secs / done * total_rows
+    if backward:
+        full_s *= 3.5  # forward (two products per pair) plus backward (five)
+    flops = tile_flops(wl, nnz) + (tile_flops(wl, nnz, True) if backward else 0)
+    return {"value": flops / full_s / 1e12, "unit": "TFLOP/s", "cores": _cores(), "kind": "oracle",
+            "sample": f"{done} query rows of head 0 (fp64 NumPy forward, {secs:.1f} s), extrapolated to "
+                      f"{total_rows} rows" + (" x3.5 for forward+backward" if backward else ""),
+            "extrapolated_ms_per_step": full_s * 1e3}
+
+
+# ---------------------------------------------------------------------------
+# the GPU arm
+# ---------------------------------------------------------------------------
+
+def run_ours(args, rank, world, local_rank):
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+
+    import block_sparse_attention_csr_b200 as rb
+    from block_sparse_attention_csr_b200 import inputs as I
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    wl = I.WORKLOADS[args.workload]
+    backward = wl.backward
+    peak, peak_sus, hbm, peak_src = _peaks()
+    stream = torch.cuda.current_stream(dev)
+
+    # mask: static, built once per shape
+    t0 = time.perf_counter()
+    csr = rb.radial_mask_build(wl.frames, wl.tokens_per_frame, wl.block, sink=1)
+    mask_ms = (time.perf_counter() - t0) * 1e3
+    t0 = time.perf_counter()
+    csr = rb.radial_mask_build(wl.frames, wl.tokens_per_frame, wl.block, sink=1)
+    mask_ms = min(mask_ms, (time.perf_counter() - t0) * 1e3)
+    nnz = rb.radial_csr_info(csr)["nnz"]
+
+    q, k, v, *rest = I.draw(wl, device=dev, backward=True)
+    do = rest[0]
+    o = torch.empty_like(q)
+    lse = torch.empty(q.shape[:3], dtype=torch.float32, device=dev)
+    if backward:
+        dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+        ws = torch.empty(rb.radial_attn_bwd_workspace_size(q), dtype=torch.uint8, device=dev)
+
+    def step():
+        rb.radial_attn_fwd(csr, q, k, v, o=o, lse=lse, stream=stream)
+        if backward:
+            rb.radial_attn_bwd(csr, do, q, k, v, o, lse, dq, dk, dv, ws, stream=stream)
+
+    for _ in range(args.warmup):
+        step()
+    rb.radial_device_status(stream)
+
+    phys = local_rank
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+    if vis:
+        try:
+            phys = int(vis.split(",")[local_rank])
+        except ValueError:
+            pass
+    sampler = ClockSampler(phys)
+
+    # ---- timed region: K steps, events on the launching stream
+    launches0 = rb.radial_launch_count()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    sampler.start()
+    time.sleep(0.3)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    for a, b in evs:
+        a.record(stream)
+        step()
+        b.record(stream)
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    clocks = sampler.stop()
+    launches = rb.radial_launch_count() - launches0
+    rb.radial_device_status(stream)
+    step_ms = [a.elapsed_time(b) for a, b in evs]
+    ms = float(np.mean(step_ms))
+    ms_max = max_over_ranks(ms, world, dev)
+
+    flops_step = tile_flops(wl, nnz) + (tile_flops(wl, nnz, True) if backward else 0)
+    value = whole_job_tflops(flops_step, world, ms_max)
+
+    # forward kernel alone (dominant kernel of the default step) for the roofline
+    fwd_ms = ms
+    if backward:
+        e = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(3)]
+        for a, b in e:
+            a.record(stream)
+            rb.radial_attn_fwd(csr, q, k, v, o=o, lse=lse, stream=stream)
+            b.record(stream)
+        torch.cuda.synchronize(dev)
+        fwd_ms = float(np.mean([a.elapsed_time(b) for a, b in e]))
+    fwd_tf = tile_flops(wl, nnz) / (fwd_ms * 1e-3) / 1e12
+
+    extra = {}
+    if rank == 0 and not args.quick:
+        # dense comparator: same kernels, all-ones mask, same shape
+        dcsr = rb.radial_mask_build_dense(wl.n, wl.block)
+        dnnz = rb.radial_csr_info(dcsr)["nnz"]
+        rb.radial_attn_fwd(dcsr, q, k, v, o=o, lse=lse, stream=stream)
+        e = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(2)]
+        for a, b in e:
+            a.record(stream)
+            rb.radial_attn_fwd(dcsr, q, k, v, o=o, lse=lse, stream=stream)
+            b.record(stream)
+        torch.cuda.synchronize(dev)
+        dense_ms = float(np.mean([a.elapsed_time(b) for a, b in e]))
+        extra["dense"] = {"fwd_ms": dense_ms, "tflops": tile_flops(wl, dnnz) / (dense_ms * 1e-3) / 1e12,
+                          "speedup_radial_vs_dense_fwd": dense_ms / fwd_ms}
+        del dcsr
+        if not backward and not args.no_bwd:
+            dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+            ws = torch.empty(rb.radial_attn_bwd_workspace_size(q), dtype=torch.uint8, device=dev)
+            rb.radial_attn_bwd(csr, do, q, k, v, o, lse, dq, dk, dv, ws, stream=stream)
+            e = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(2)]
+            for a, b in e:
+                a.record(stream)
+                rb.radial_attn_bwd(csr, do, q, k, v, o, lse, dq, dk, dv, ws, stream=stream)
+                b.record(stream)
+            torch.cuda.synchronize(dev)
+            bwd_ms = float(np.mean([a.elapsed_time(b) for a, b in e]))
+            extra["bwd"] = {"ms": bwd_ms, "tflops_algorithmic": tile_flops(wl, nnz, True) / (bwd_ms * 1e-3) / 1e12,
+                            "note": "10*B^2*d flops per tile (5 GEMMs); the kernels issue 7 (dQ pass recomputes S, dP)"}
+            del dq, dk, dv, ws
+
+    # ---- end to end through the public API with host buffers
+    e2e = None
+    if rank == 0 and not args.quick:
+        hq, hk, hv = (t.cpu().pin_memory() for t in (q, k, v))
+        hdo = do.cpu().pin_memory() if backward else None
+        ho = torch.empty(q.shape, dtype=torch.bfloat16).pin_memory()
+        hl = torch.empty(q.shape[:3], dtype=torch.float32).pin_memory()
+        if backward:
+            hdq = torch.empty(q.shape, dtype=torch.bfloat16).pin_memory()
+            hdk, hdv = torch.empty_like(hdq).pin_memory(), torch.empty_like(hdq).pin_memory()
+
+        def e2e_step():
+            q.copy_(hq, non_blocking=True)
+            k.copy_(hk, non_blocking=True)
+            v.copy_(hv, non_blocking=True)
+            if backward:
+                do.copy_(hdo, non_blocking=True)
+            rb.radial_attn_fwd(csr, q, k, v, o=o, lse=lse, stream=stream)
+            if backward:
+                rb.radial_attn_bwd(csr, do, q, k, v, o, lse, dq, dk, dv, ws, stream=stream)
+                hdq.copy_(dq, non_blocking=True)
+                hdk.copy_(dk, non_blocking=True)
+                hdv.copy_(dv, non_blocking=True)
+            ho.copy_(o, non_blocking=True)
+            hl.copy_(lse, non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize(dev)
+        n_e2e = max(2, min(5, args.steps))
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(n_e2e):
+            e2e_step()
+        b.record(stream)
+        torch.cuda.synchronize(dev)
+        e2e_ms = a.elapsed_time(b) / n_e2e
+        elt = q.numel() * 2
+        h2d = 3 * elt + (elt if backward else 0)
+        d2h = elt + lse.numel() * 4 + (3 * elt if backward else 0)
+        e2e = {"value": flops_step / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": e2e_ms,
+               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+               "path": "pinned host -> device copies, radial_attn_fwd%s via the C ABI, device -> host result copies"
+                       % ("/bwd" if backward else "")}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(wl, nnz, q, k, v, budget_s=args.cpu_budget, backward=backward)
+
+    if rank == 0:
+        traffic = None
+        tp = os.path.join(ROOT, "profiles", "fwd_traffic.json")
+        if os.path.exists(tp):
+            try:
+                with open(tp) as fh:
+                    tj = json.load(fh)
+                if tj.get("workload") == wl.name and tj.get("kernel_sha") == kernel_sha():
+                    traffic = tj.get("dram_bytes_per_launch")
+            except Exception:
+                traffic = None
+        line = {
+            "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_max, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded N(0,1) bf16 Q,K,V%s)" % (",dO" if backward else ""),
+            "config": config_of(wl, nnz),
+            "pct_of_tensor_peak": 100.0 * value / world / peak,
+            "mask_build_ms": mask_ms,
+            "roofline": {"bound": "tensor", "kernel": "radial_fwd_kernel<128>", "achieved": fwd_tf, "peak": peak,
+                         "unit": "TFLOP/s", "frac": fwd_tf / peak, "peak_source": f"{peak_src} bf16 burst",
+                         "frac_of_sustained": fwd_tf / peak_sus, "traffic": traffic,
+                         "algorithmic_flops_per_launch": tile_flops(wl, nnz), "launch_ms": fwd_ms},
+            "cpu_baseline": cpu,
+            "e2e": e2e,
+            "gpu_launches": int(launches),
+            "clocks": clocks,
+        }
+        line.update(extra)
+        print(json.dumps(line), flush=True)
+
+
+def kernel_sha():
+    import hashlib
+    h = hashlib.sha1()
+    for f in ("attn_fwd.cuh", "sm100_primitives.cuh", "mask_build.cuh"):
+        with open(os.path.join(ROOT, "block_sparse_attention_csr_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:12]
+
+
+# ---------------------------------------------------------------------------
+# the reference arm: the CPU reference as it stands, on the host cores
+# ---------------------------------------------------------------------------
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return
+    import numpy as np
+    import torch
+    from block_sparse_attention_csr_b200 import inputs as I
+    from oracle import attention as A
+    from oracle import mask as M
+
+    wl = I.WORKLOADS[args.workload]
+    st = M.tile_states_intervals(wl.frames, wl.tokens_per_frame, wl.block, True)
+    nnz = int((st != 0).sum())
+    # one head's K, V drawn on the CPU with the same recipe's generator
+    g = torch.Generator(device="cpu").manual_seed(wl.seed)
+    shape = (wl.n, wl.head_dim)
+    q = torch.randn(shape, generator=g).mul_(wl.value_scale).to(torch.bfloat16).double().numpy()
+    k = torch.randn(shape, generator=g).mul_(wl.value_scale).to(torch.bfloat16).double().numpy()
+    v = torch.randn(shape, generator=g).mul_(wl.value_scale).to(torch.bfloat16).double().numpy()
+    rows_per_step = args.ref_rows
+    rng = np.random.default_rng(9)
+    times = []
+    for s in range(args.warmup + args.steps):
+        rows = np.sort(rng.choice(wl.n, rows_per_step, replace=False))
+        t0 = time.perf_counter()
+        A.forward_rows(q, k, v, rows, wl.frames, wl.tokens_per_frame, True)
+        dt = time.perf_counter() - t0
+        if s >= args.warmup:
+            times.append(dt)
+    per_row = float(np.mean(times)) / rows_per_step
+    full_s = per_row * wl.batch * wl.heads * wl.n
+    if wl.backward:
+        full_s *= 3.5
+    flops = tile_flops(wl, nnz) + (tile_flops(wl, nnz, True) if wl.backward else 0)
+    value = flops / full_s / 1e12
+    sample = (f"{rows_per_step} query rows of one head per step (fp64 NumPy), extrapolated to "
+              f"{wl.batch * wl.heads * wl.n} rows" + (" x3.5 for forward+backward" if wl.backward else ""))
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": full_s * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": config_of(wl, nnz),
+            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": _cores(), "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="hunyuan720p")
+    ap.add_argument("--quick", action="store_true", help="skip dense, e2e and extras")
+    ap.add_argument("--no-bwd", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=15.0)
+    ap.add_argument("--ref-rows", type=int, default=512)
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "ours":
+        args.warmup = 3
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+    if world > 1:
+        import datetime
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        run_ours(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -22,6 +22,7 @@ from ._binding import (  # noqa: F401
     radial_mask_build,
     radial_mask_build_dense,
     radial_params_default,
+    radial_selftest_bounded_wait,
 )
 
 TILE_FULL = 1

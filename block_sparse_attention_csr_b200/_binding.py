@@ -27,7 +27,7 @@ EXPORTED = (
     "radial_params_default", "radial_mask_build", "radial_mask_build_dense", "radial_csr_info",
     "radial_csr_copy_to_host", "radial_csr_free", "radial_attn_fwd",
     "radial_attn_bwd_workspace_size", "radial_attn_bwd", "radial_device_status",
-    "radial_status_str", "radial_last_error", "radial_launch_count",
+    "radial_status_str", "radial_last_error", "radial_launch_count", "radial_selftest_bounded_wait",
 )
 
 
@@ -97,6 +97,8 @@ def load(path=None):
         L.radial_status_str.restype = ctypes.c_char_p
         L.radial_last_error.argtypes = []
         L.radial_last_error.restype = ctypes.c_char_p
+        L.radial_selftest_bounded_wait.argtypes = [ctypes.c_uint32, vp]
+        L.radial_selftest_bounded_wait.restype = ctypes.c_int
         L.radial_launch_count.argtypes = []
         L.radial_launch_count.restype = i64
         _lib = L
@@ -252,6 +254,10 @@ def radial_attn_bwd(csr, do, q, k, v, o, lse, dq=None, dk=None, dv=None, workspa
 
 def radial_device_status(stream=None):
     _check(load().radial_device_status(_stream(stream)), "radial_device_status")
+
+
+def radial_selftest_bounded_wait(limit_ms=20, stream=None):
+    _check(load().radial_selftest_bounded_wait(int(limit_ms), _stream(stream)), "radial_selftest_bounded_wait")
 
 
 def radial_launch_count():

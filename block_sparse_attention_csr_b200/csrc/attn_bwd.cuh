@@ -1,2 +1,624 @@
-// Block-sparse backward of Radial Attention on sm_100a (see radial_lib.cu).
+// Block-sparse backward of Radial Attention on sm_100a.
+//
+// Gradients of O = softmax(Q K^T * scale + M) V (the sparse-attention
+// equation, Eq.2, of the Radial Attention review on jaehun.me, §3) with
+// respect to Q, K and V, as the LoRA length-extension fine-tuning of §4.3
+// back-propagates through every radial attention layer.  With
+// P = exp(S*scale - LSE) (S = Q K^T, masked), Dr = rowsum(dO o O):
+//   dV = P^T dO,   dP = dO V^T,   dS = P o (dP - Dr),
+//   dK = scale * dS^T Q,          dQ = scale * dS K.
+// Only the mask's active 128x128 tiles are visited (§4.2, block-wise).
+//
+// Three kernels, no atomics, deterministic:
+//  1. bwd_rowdot:  Dr[row] = sum_d dO*O (fp32, into the caller's workspace).
+//  2. bwd_dkdv:    one work item per (batch*head, 128-key tile); walks the
+//                  query tiles of the mask's CSC column: S^T = K Q^T and
+//                  dP^T = V dO^T into TMEM; one thread per key row forms P^T
+//                  and dS^T (bf16, written back over the consumed S^T / dP^T
+//                  columns); dV += P^T dO and dK += dS^T Q accumulate in TMEM
+//                  with P^T / dS^T as the TMEM A operand.
+//  3. bwd_dq:      one work item per (batch*head, 128-query tile); walks the
+//                  CSR row: S = Q K^T, dP = dO V^T into TMEM; one thread per
+//                  query row forms dS (bf16, TMEM); dQ += dS K in TMEM.
+// Recomputing S and dP in (3) costs 2 extra GEMMs per tile (7 instead of 5)
+// and removes the fp32 dQ atomics a single fused pass would need.
 #pragma once
+
+#include <cstdint>
+#include <cuda_bf16.h>
+
+#include "attn_fwd.cuh"
+#include "mask_build.cuh"
+#include "sm100_primitives.cuh"
+
+namespace radial {
+
+// ---------------------------------------------------------------------------
+// 1. Dr = rowsum(dO o O)
+// ---------------------------------------------------------------------------
+template <int D>
+__global__ void bwd_rowdot_kernel(const __nv_bfloat16* __restrict__ dO, const __nv_bfloat16* __restrict__ O,
+                                  int heads, int n, int64_t sb, int64_t sh, int64_t sn,
+                                  int64_t rows, float* __restrict__ dr) {
+  // 16 threads per row, 8 bf16 (16 bytes) per thread per step
+  constexpr int TPR = 16;
+  const int64_t row = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) / TPR;
+  const int sub = threadIdx.x % TPR;
+  float acc = 0.f;
+  if (row < rows) {
+    const int64_t bh = row / n;
+    const int a = static_cast<int>(row - bh * n);
+    const int b = static_cast<int>(bh / heads), h = static_cast<int>(bh - static_cast<int64_t>(b) * heads);
+    const int64_t off = b * sb + h * sh + a * sn;
+#pragma unroll
+    for (int c = sub * 8; c < D; c += TPR * 8) {
+      const uint4 x = *reinterpret_cast<const uint4*>(dO + off + c);
+      const uint4 y = *reinterpret_cast<const uint4*>(O + off + c);
+      const __nv_bfloat162* xp = reinterpret_cast<const __nv_bfloat162*>(&x);
+      const __nv_bfloat162* yp = reinterpret_cast<const __nv_bfloat162*>(&y);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float2 xf = __bfloat1622float2(xp[e]);
+        const float2 yf = __bfloat1622float2(yp[e]);
+        acc = fmaf(xf.x, yf.x, acc);
+        acc = fmaf(xf.y, yf.y, acc);
+      }
+    }
+  }
+#pragma unroll
+  for (int o = TPR / 2; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+  if (row < rows && sub == 0) dr[row] = acc;
+}
+
+struct BwdParams {
+  // 128-token tile plan: CSR (query-major) and CSC (key-major)
+  const int32_t* row_ptr;
+  const int32_t* col_idx;
+  const uint8_t* kind;
+  const int32_t* row_order;
+  const int32_t* col_ptr;
+  const int32_t* row_idx;
+  const uint8_t* kind_t;
+  const int32_t* col_order;
+  int32_t nt;
+  int32_t f, s, n, sink;
+  int32_t heads, items;
+  int64_t sb, sh, sn;  // element strides shared by all bf16 tensors
+  const float* lse;    // [B, H, N]
+  const float* dr;     // [B, H, N]
+  __nv_bfloat16* dq;
+  __nv_bfloat16* dk;
+  __nv_bfloat16* dv;
+  float scale;
+  float scale_log2;
+};
+
+// Allowed query rows (relative to a0, 128 wide) of key token b = j*s + l:
+// the transpose of row_mask_bits.
+__device__ __forceinline__ void col_mask_bits(int f_unused, int s, int n, int sink, int j, int l, int a0,
+                                              uint32_t (&mw)[4]) {
+  (void)f_unused;
+  mw[0] = mw[1] = mw[2] = mw[3] = 0u;
+  const int aend = min(a0 + 128, n);
+  for (int i = a0 / s; i * s < aend; ++i) {
+    const int seg_lo = max(a0, i * s) - a0;
+    const int seg_hi = min(aend, (i + 1) * s) - 1 - a0;
+    int lo, hi;
+    if (sink && j == 0) {
+      lo = seg_lo;
+      hi = seg_hi;
+    } else {
+      const int d = i > j ? i - j : j - i;
+      const int r = 31 - __clz(d > 1 ? d : 1);
+      const int h = (s >> r) - 1;
+      const int center = i * s + l - a0;
+      if (h >= 0) {
+        lo = max(seg_lo, center - h);
+        hi = min(seg_hi, center + h);
+      } else {
+        const long long period = ((1LL << r) + s - 1) / s;
+        if (d % period != 0) continue;
+        lo = max(seg_lo, center);
+        hi = min(seg_hi, center);
+      }
+    }
+    if (lo <= hi) set_bits(mw, lo, hi);
+  }
+}
+
+template <int D>
+struct BwdCfg {
+  static constexpr int TILE_BYTES = 128 * D * 2;
+  static constexpr int NBOX = D / 64;
+  static constexpr int STAGES = 2;
+  // smem: fixed pair (2 tiles) + STAGES x streamed pair (2 tiles each)
+  static constexpr int SMEM_FIX = 0;
+  static constexpr int SMEM_STREAM = 2 * TILE_BYTES;
+  static constexpr int SMEM_VEC = SMEM_STREAM + STAGES * 2 * TILE_BYTES;  // 2 x 2 x 128 floats
+  static constexpr int SMEM_BAR = SMEM_VEC + 2 * 2 * 128 * 4;
+  static constexpr int SMEM_BYTES = SMEM_BAR + 256 + 1024;
+};
+
+struct BwdBars {
+  uint64_t fix_full, fix_empty, acc_empty, mma_done;
+  uint64_t s_full, s_free, ew_full[2], mma2_done[2];
+  uint64_t st_full[2], st_empty[2];
+  uint32_t tmem_base;
+  int abort;
+};
+
+__device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
+// ---------------------------------------------------------------------------
+// 2. dK, dV: key-major walk of the CSC
+// ---------------------------------------------------------------------------
+// TMEM: dK [0,D) dV [128,128+D) S^T [256,384) dP^T [384,512);
+// P^T (bf16) overwrites S^T columns [256,320), dS^T overwrites [384,448).
+template <int D>
+__global__ void __launch_bounds__(192, 1)
+    radial_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                           const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
+                           const BwdParams p) {
+  using C = BwdCfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint8_t* sK = smem + C::SMEM_FIX;
+  uint8_t* sV = sK + C::TILE_BYTES;
+  uint8_t* sQ = smem + C::SMEM_STREAM;                 // stage st: sQ + st*2*TILE
+  float* sVec = reinterpret_cast<float*>(smem + C::SMEM_VEC);  // [2 buf][lse2 | dr][128]
+  BwdBars* bars = reinterpret_cast<BwdBars*>(smem + C::SMEM_BAR);
+  volatile int* abort_flag = &bars->abort;
+  constexpr uint32_t TM_DK = 0, TM_DV = 128, TM_S = 256, TM_DP = 384;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    bars->abort = 0;
+    mbar_init(&bars->fix_full, 1);
+    mbar_init(&bars->fix_empty, 1);
+    mbar_init(&bars->acc_empty, 128);
+    mbar_init(&bars->mma_done, 1);
+    mbar_init(&bars->s_full, 1);
+    mbar_init(&bars->s_free, 128);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&bars->ew_full[b], 128);
+      mbar_init(&bars->mma2_done[b], 1);
+      mbar_init(&bars->st_full[b], 1);
+      mbar_init(&bars->st_empty[b], 1);
+    }
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(&bars->tmem_base, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bars->tmem_base;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      uint32_t it = 0, item_i = 0;
+      for (int item = blockIdx.x; item < p.items; item += gridDim.x, ++item_i) {
+        const int bh = item / p.nt;
+        const int u = p.col_order[item - bh * p.nt];
+        const int b = bh / p.heads, h = bh - b * p.heads;
+        if (item_i > 0) mbar_wait(&bars->fix_empty, (item_i - 1) & 1, abort_flag);
+        mbar_arrive_expect_tx(&bars->fix_full, 2 * C::TILE_BYTES);
+#pragma unroll
+        for (int x = 0; x < C::NBOX; ++x) {
+          tma_load_4d(sK + x * 16384, &tmK, &bars->fix_full, x * 64, u * 128, h, b);
+          tma_load_4d(sV + x * 16384, &tmV, &bars->fix_full, x * 64, u * 128, h, b);
+        }
+        for (int q = p.col_ptr[u]; q < p.col_ptr[u + 1]; ++q, ++it) {
+          const int t = p.row_idx[q];
+          const uint32_t st = it % C::STAGES, use = it / C::STAGES;
+          if (use > 0) mbar_wait(&bars->st_empty[st], (use - 1) & 1, abort_flag);
+          uint8_t* dstQ = sQ + st * 2 * C::TILE_BYTES;
+          uint8_t* dstO = dstQ + C::TILE_BYTES;
+          mbar_arrive_expect_tx(&bars->st_full[st], 2 * C::TILE_BYTES);
+#pragma unroll
+          for (int x = 0; x < C::NBOX; ++x) {
+            tma_load_4d(dstQ + x * 16384, &tmQ, &bars->st_full[st], x * 64, t * 128, h, b);
+            tma_load_4d(dstO + x * 16384, &tmdO, &bars->st_full[st], x * 64, t * 128, h, b);
+          }
+        }
+      }
+      for (uint32_t k = (it > C::STAGES ? it - C::STAGES : 0); k < it; ++k)
+        mbar_wait_drain(&bars->st_full[k % C::STAGES], (k / C::STAGES) & 1);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t idesc_s = idesc_bf16_f32(128, 128, false, false);
+      constexpr uint32_t idesc_g = idesc_bf16_f32(128, D, false, true);
+      const uint32_t k_base = smem_u32(sK), v_base = smem_u32(sV), q_base = smem_u32(sQ);
+      uint32_t it = 0, item_i = 0;
+      for (int item = blockIdx.x; item < p.items; item += gridDim.x, ++item_i) {
+        const int bh = item / p.nt;
+        const int u = p.col_order[item - bh * p.nt];
+        const uint32_t n_tiles = static_cast<uint32_t>(p.col_ptr[u + 1] - p.col_ptr[u]);
+        mbar_wait(&bars->fix_full, item_i & 1, abort_flag);
+        tc_fence_after();
+        for (uint32_t j = 0; j < n_tiles; ++j) {
+          const uint32_t g = it + j, st = g % C::STAGES;
+          mbar_wait(&bars->st_full[st], (g / C::STAGES) & 1, abort_flag);
+          // S^T / dP^T columns still hold P^T / dS^T of the previous tile until
+          // its dV / dK MMAs have completed.
+          if (g >= 1) mbar_wait(&bars->mma2_done[(g - 1) & 1], ((g - 1) >> 1) & 1, abort_flag);
+          tc_fence_after();
+          const uint32_t qb = q_base + st * 2 * C::TILE_BYTES, ob = qb + C::TILE_BYTES;
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+            mma_ss(tmem + TM_S, smem_desc(k_base + off, 16, 1024, kSwizzle128B),
+                   smem_desc(qb + off, 16, 1024, kSwizzle128B), idesc_s, kk > 0 ? 1u : 0u);
+          }
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+            mma_ss(tmem + TM_DP, smem_desc(v_base + off, 16, 1024, kSwizzle128B),
+                   smem_desc(ob + off, 16, 1024, kSwizzle128B), idesc_s, kk > 0 ? 1u : 0u);
+          }
+          mma_commit(&bars->s_full);
+          mbar_wait(&bars->ew_full[g & 1], (g >> 1) & 1, abort_flag);
+          if (j == 0 && item_i > 0) mbar_wait(&bars->acc_empty, (item_i - 1) & 1, abort_flag);
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk) {  // K = 128 query rows, 16 per MMA
+            mma_ts(tmem + TM_DV, tmem + TM_S + kk * 8, smem_desc(ob + kk * 2048, 16384, 1024, kSwizzle128B),
+                   idesc_g, (j > 0 || kk > 0) ? 1u : 0u);
+          }
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk) {
+            mma_ts(tmem + TM_DK, tmem + TM_DP + kk * 8, smem_desc(qb + kk * 2048, 16384, 1024, kSwizzle128B),
+                   idesc_g, (j > 0 || kk > 0) ? 1u : 0u);
+          }
+          mma_commit(&bars->mma2_done[g & 1]);
+          mma_commit(&bars->st_empty[st]);
+          if (j + 1 == n_tiles) mma_commit(&bars->fix_empty);
+        }
+        it += n_tiles;
+      }
+      mma_commit(&bars->mma_done);
+      mbar_wait_drain(&bars->mma_done, 0);
+    }
+  } else {
+    const int quarter = warp & 3;
+    const int row = quarter * 32 + lane;
+    const int tid = threadIdx.x - 64;  // 0..127 inside the warpgroup
+    const uint32_t lane_addr = static_cast<uint32_t>(quarter * 32) << 16;
+    constexpr float kLog2e = 1.4426950408889634f;
+    uint32_t it = 0, item_i = 0;
+    for (int item = blockIdx.x; item < p.items; item += gridDim.x, ++item_i) {
+      const int bh = item / p.nt;
+      const int u = p.col_order[item - bh * p.nt];
+      const int b = bh / p.heads, h = bh - b * p.heads;
+      const int key = u * 128 + row;
+      const bool valid = key < p.n;
+      const int kj = valid ? key / p.s : 0;
+      const int kl = valid ? key - kj * p.s : 0;
+      const int c0 = p.col_ptr[u];
+      const uint32_t n_tiles = static_cast<uint32_t>(p.col_ptr[u + 1] - c0);
+      const float* lse_bh = p.lse + static_cast<int64_t>(bh) * p.n;
+      const float* dr_bh = p.dr + static_cast<int64_t>(bh) * p.n;
+      for (uint32_t j = 0; j < n_tiles; ++j) {
+        const uint32_t g = it + j;
+        const int t = p.row_idx[c0 + j];
+        const bool partial = p.kind_t[c0 + j] != kTileFull;
+        // per-query statistics of this query tile -> shared memory
+        float* vbuf = sVec + (g & 1) * 256;
+        {
+          const int a = t * 128 + tid;
+          vbuf[tid] = a < p.n ? lse_bh[a] * kLog2e : INFINITY;
+          vbuf[128 + tid] = a < p.n ? dr_bh[a] : 0.f;
+        }
+        named_bar_sync(1, 128);
+        uint32_t mw[4] = {0xffffffffu, 0xffffffffu, 0xffffffffu, 0xffffffffu};
+        if (partial) {
+          if (valid)
+            col_mask_bits(p.f, p.s, p.n, p.sink, kj, kl, t * 128, mw);
+          else
+            mw[0] = mw[1] = mw[2] = mw[3] = 0u;
+        }
+        mbar_wait(&bars->s_full, g & 1, abort_flag);
+        __syncwarp();
+        tc_fence_after();
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          uint32_t rs[32], rp[32];
+          tmem_ld32(tmem + lane_addr + TM_S + c * 32, rs);
+          tmem_ld32(tmem + lane_addr + TM_DP + c * 32, rp);
+          tmem_wait_ld();
+          uint32_t pw[16], dw[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            float pv[2], dv[2];
+#pragma unroll
+            for (int z = 0; z < 2; ++z) {
+              const int qi = c * 32 + 2 * e + z;
+              const bool ok = (mw[qi >> 5] >> (qi & 31)) & 1u;
+              const float x = fmaf(__uint_as_float(rs[2 * e + z]), p.scale_log2, -vbuf[qi]);
+              pv[z] = ok ? ex2_approx(x) : 0.f;
+              dv[z] = pv[z] * (__uint_as_float(rp[2 * e + z]) - vbuf[128 + qi]);
+            }
+            pw[e] = pack_bf16x2(pv[0], pv[1]);
+            dw[e] = pack_bf16x2(dv[0], dv[1]);
+          }
+          tmem_st16(tmem + lane_addr + TM_S + c * 16, pw);
+          tmem_st16(tmem + lane_addr + TM_DP + c * 16, dw);
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(&bars->ew_full[g & 1]);
+      }
+      // epilogue: dK (scaled), dV
+      const uint32_t g_last = it + n_tiles - 1;
+      mbar_wait(&bars->mma2_done[g_last & 1], (g_last >> 1) & 1, abort_flag);
+      __syncwarp();
+      tc_fence_after();
+      const int64_t off = static_cast<int64_t>(b) * p.sb + static_cast<int64_t>(h) * p.sh +
+                          static_cast<int64_t>(valid ? key : 0) * p.sn;
+#pragma unroll
+      for (int which = 0; which < 2; ++which) {
+        const uint32_t col = which == 0 ? TM_DK : TM_DV;
+        const float mul = which == 0 ? p.scale : 1.0f;
+        __nv_bfloat16* dst = (which == 0 ? p.dk : p.dv) + off;
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t r[32];
+          tmem_ld32(tmem + lane_addr + col + c * 32, r);
+          tmem_wait_ld();
+          if (valid) {
+            uint32_t pk[16];
+#pragma unroll
+            for (int e = 0; e < 16; ++e)
+              pk[e] = pack_bf16x2(__uint_as_float(r[2 * e]) * mul, __uint_as_float(r[2 * e + 1]) * mul);
+            uint4* o4 = reinterpret_cast<uint4*>(dst + c * 32);
+#pragma unroll
+            for (int v = 0; v < 4; ++v) o4[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&bars->acc_empty);
+      it += n_tiles;
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// 3. dQ: query-major walk of the CSR
+// ---------------------------------------------------------------------------
+// TMEM: S [0,128) dP [128,256) dQ [256,256+D) dS0 [384,448) dS1 [448,512).
+template <int D>
+__global__ void __launch_bounds__(192, 1)
+    radial_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                         const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
+                         const BwdParams p) {
+  using C = BwdCfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint8_t* sQ = smem + C::SMEM_FIX;
+  uint8_t* sdO = sQ + C::TILE_BYTES;
+  uint8_t* sK = smem + C::SMEM_STREAM;  // stage st: sK + st*2*TILE, V follows K
+  BwdBars* bars = reinterpret_cast<BwdBars*>(smem + C::SMEM_BAR);
+  volatile int* abort_flag = &bars->abort;
+  constexpr uint32_t TM_S = 0, TM_DP = 128, TM_DQ = 256, TM_DS = 384;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    bars->abort = 0;
+    mbar_init(&bars->fix_full, 1);
+    mbar_init(&bars->fix_empty, 1);
+    mbar_init(&bars->acc_empty, 128);
+    mbar_init(&bars->mma_done, 1);
+    mbar_init(&bars->s_full, 1);
+    mbar_init(&bars->s_free, 128);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&bars->ew_full[b], 128);
+      mbar_init(&bars->mma2_done[b], 1);
+      mbar_init(&bars->st_full[b], 1);
+      mbar_init(&bars->st_empty[b], 1);
+    }
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(&bars->tmem_base, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bars->tmem_base;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      uint32_t it = 0, item_i = 0;
+      for (int item = blockIdx.x; item < p.items; item += gridDim.x, ++item_i) {
+        const int bh = item / p.nt;
+        const int t = p.row_order[item - bh * p.nt];
+        const int b = bh / p.heads, h = bh - b * p.heads;
+        if (item_i > 0) mbar_wait(&bars->fix_empty, (item_i - 1) & 1, abort_flag);
+        mbar_arrive_expect_tx(&bars->fix_full, 2 * C::TILE_BYTES);
+#pragma unroll
+        for (int x = 0; x < C::NBOX; ++x) {
+          tma_load_4d(sQ + x * 16384, &tmQ, &bars->fix_full, x * 64, t * 128, h, b);
+          tma_load_4d(sdO + x * 16384, &tmdO, &bars->fix_full, x * 64, t * 128, h, b);
+        }
+        for (int q = p.row_ptr[t]; q < p.row_ptr[t + 1]; ++q, ++it) {
+          const int kb = p.col_idx[q];
+          const uint32_t st = it % C::STAGES, use = it / C::STAGES;
+          if (use > 0) mbar_wait(&bars->st_empty[st], (use - 1) & 1, abort_flag);
+          uint8_t* dK = sK + st * 2 * C::TILE_BYTES;
+          uint8_t* dV = dK + C::TILE_BYTES;
+          mbar_arrive_expect_tx(&bars->st_full[st], 2 * C::TILE_BYTES);
+#pragma unroll
+          for (int x = 0; x < C::NBOX; ++x) {
+            tma_load_4d(dK + x * 16384, &tmK, &bars->st_full[st], x * 64, kb * 128, h, b);
+            tma_load_4d(dV + x * 16384, &tmV, &bars->st_full[st], x * 64, kb * 128, h, b);
+          }
+        }
+      }
+      for (uint32_t k = (it > C::STAGES ? it - C::STAGES : 0); k < it; ++k)
+        mbar_wait_drain(&bars->st_full[k % C::STAGES], (k / C::STAGES) & 1);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t idesc_s = idesc_bf16_f32(128, 128, false, false);
+      constexpr uint32_t idesc_g = idesc_bf16_f32(128, D, false, true);
+      const uint32_t q_base = smem_u32(sQ), o_base = smem_u32(sdO), k_base = smem_u32(sK);
+      uint32_t it = 0, item_i = 0;
+      auto issue_dq = [&](uint32_t g, uint32_t j) {
+        const uint32_t st = g % C::STAGES, db = g & 1;
+        mbar_wait(&bars->ew_full[db], (g >> 1) & 1, abort_flag);
+        if (j == 0 && item_i > 0) mbar_wait(&bars->acc_empty, (item_i - 1) & 1, abort_flag);
+        tc_fence_after();
+        const uint32_t kb = k_base + st * 2 * C::TILE_BYTES;
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          mma_ts(tmem + TM_DQ, tmem + TM_DS + db * 64 + kk * 8,
+                 smem_desc(kb + kk * 2048, 16384, 1024, kSwizzle128B), idesc_g, (j > 0 || kk > 0) ? 1u : 0u);
+        mma_commit(&bars->mma2_done[db]);
+        mma_commit(&bars->st_empty[st]);
+      };
+      for (int item = blockIdx.x; item < p.items; item += gridDim.x, ++item_i) {
+        const int bh = item / p.nt;
+        const int t = p.row_order[item - bh * p.nt];
+        const uint32_t n_tiles = static_cast<uint32_t>(p.row_ptr[t + 1] - p.row_ptr[t]);
+        mbar_wait(&bars->fix_full, item_i & 1, abort_flag);
+        tc_fence_after();
+        for (uint32_t j = 0; j < n_tiles; ++j) {
+          const uint32_t g = it + j, st = g % C::STAGES;
+          mbar_wait(&bars->st_full[st], (g / C::STAGES) & 1, abort_flag);
+          if (g >= 1) mbar_wait(&bars->s_free, (g - 1) & 1, abort_flag);
+          tc_fence_after();
+          const uint32_t kb = k_base + st * 2 * C::TILE_BYTES, vb = kb + C::TILE_BYTES;
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+            mma_ss(tmem + TM_S, smem_desc(q_base + off, 16, 1024, kSwizzle128B),
+                   smem_desc(kb + off, 16, 1024, kSwizzle128B), idesc_s, kk > 0 ? 1u : 0u);
+          }
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+            mma_ss(tmem + TM_DP, smem_desc(o_base + off, 16, 1024, kSwizzle128B),
+                   smem_desc(vb + off, 16, 1024, kSwizzle128B), idesc_s, kk > 0 ? 1u : 0u);
+          }
+          mma_commit(&bars->s_full);
+          if (j + 1 == n_tiles) mma_commit(&bars->fix_empty);
+          if (j > 0) issue_dq(g - 1, j - 1);
+        }
+        issue_dq(it + n_tiles - 1, n_tiles - 1);
+        it += n_tiles;
+      }
+      mma_commit(&bars->mma_done);
+      mbar_wait_drain(&bars->mma_done, 0);
+    }
+  } else {
+    const int quarter = warp & 3;
+    const int row = quarter * 32 + lane;
+    const uint32_t lane_addr = static_cast<uint32_t>(quarter * 32) << 16;
+    constexpr float kLog2e = 1.4426950408889634f;
+    uint32_t it = 0, item_i = 0;
+    for (int item = blockIdx.x; item < p.items; item += gridDim.x, ++item_i) {
+      const int bh = item / p.nt;
+      const int t = p.row_order[item - bh * p.nt];
+      const int b = bh / p.heads, h = bh - b * p.heads;
+      const int a = t * 128 + row;
+      const bool valid = a < p.n;
+      const int qi = valid ? a / p.s : 0;
+      const int qk = valid ? a - qi * p.s : 0;
+      const float lse2 = valid ? p.lse[static_cast<int64_t>(bh) * p.n + a] * kLog2e : INFINITY;
+      const float drow = valid ? p.dr[static_cast<int64_t>(bh) * p.n + a] : 0.f;
+      const int p0 = p.row_ptr[t];
+      const uint32_t n_tiles = static_cast<uint32_t>(p.row_ptr[t + 1] - p0);
+      for (uint32_t j = 0; j < n_tiles; ++j) {
+        const uint32_t g = it + j, db = g & 1;
+        const int kb = p.col_idx[p0 + j];
+        const bool partial = p.kind[p0 + j] != kTileFull;
+        uint32_t mw[4] = {0xffffffffu, 0xffffffffu, 0xffffffffu, 0xffffffffu};
+        if (partial) {
+          mw[0] = mw[1] = mw[2] = mw[3] = 0u;
+          if (valid) row_mask_bits(FwdParams{nullptr, nullptr, nullptr, nullptr, 0, p.f, p.s, p.n, p.sink},
+                                   qi, qk, kb * 128, mw);
+        }
+        // dS buffer db was read by the dQ MMA of tile g-2
+        if (g >= 2) {
+          mbar_wait(&bars->mma2_done[db], ((g >> 1) - 1) & 1, abort_flag);
+          __syncwarp();
+        }
+        mbar_wait(&bars->s_full, g & 1, abort_flag);
+        __syncwarp();
+        tc_fence_after();
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          uint32_t rs[32], rp[32];
+          tmem_ld32(tmem + lane_addr + TM_S + c * 32, rs);
+          tmem_ld32(tmem + lane_addr + TM_DP + c * 32, rp);
+          tmem_wait_ld();
+          uint32_t dw[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            float dv[2];
+#pragma unroll
+            for (int z = 0; z < 2; ++z) {
+              const int ci = c * 32 + 2 * e + z;
+              const bool ok = (mw[ci >> 5] >> (ci & 31)) & 1u;
+              const float pv = ok ? ex2_approx(fmaf(__uint_as_float(rs[2 * e + z]), p.scale_log2, -lse2)) : 0.f;
+              dv[z] = pv * (__uint_as_float(rp[2 * e + z]) - drow);
+            }
+            dw[e] = pack_bf16x2(dv[0], dv[1]);
+          }
+          tmem_st16(tmem + lane_addr + TM_DS + db * 64 + c * 16, dw);
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(&bars->s_free);
+        mbar_arrive(&bars->ew_full[db]);
+      }
+      const uint32_t g_last = it + n_tiles - 1;
+      mbar_wait(&bars->mma2_done[g_last & 1], (g_last >> 1) & 1, abort_flag);
+      __syncwarp();
+      tc_fence_after();
+      __nv_bfloat16* dst = p.dq + static_cast<int64_t>(b) * p.sb + static_cast<int64_t>(h) * p.sh +
+                           static_cast<int64_t>(valid ? a : 0) * p.sn;
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t r[32];
+        tmem_ld32(tmem + lane_addr + TM_DQ + c * 32, r);
+        tmem_wait_ld();
+        if (valid) {
+          uint32_t pk[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e)
+            pk[e] = pack_bf16x2(__uint_as_float(r[2 * e]) * p.scale, __uint_as_float(r[2 * e + 1]) * p.scale);
+          uint4* o4 = reinterpret_cast<uint4*>(dst + c * 32);
+#pragma unroll
+          for (int v = 0; v < 4; ++v) o4[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&bars->acc_empty);
+      it += n_tiles;
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+}  // namespace radial

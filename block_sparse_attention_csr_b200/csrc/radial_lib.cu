@@ -23,6 +23,25 @@
 
 using namespace radial;
 
+namespace radial {
+// Failure-detection self-test: one warp waits on an mbarrier that nothing
+// will ever complete, with a short limit; the bounded wait must give up,
+// set the library's error word and let the kernel return normally.
+__global__ void selftest_bounded_wait_kernel(uint64_t limit_ns, int* waited_out) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_s;
+  if (threadIdx.x == 0) {
+    abort_s = 0;
+    mbar_init(&bar, 1);
+    fence_barrier_init();
+  }
+  __syncthreads();
+  const bool ok = mbar_wait_limit(&bar, 0, &abort_s, limit_ns);
+  __syncwarp();
+  if (threadIdx.x == 0) *waited_out = ok ? 0 : 1;
+}
+}  // namespace radial
+
 // ---------------------------------------------------------------------------
 // errors and instrumentation
 // ---------------------------------------------------------------------------
@@ -378,6 +397,62 @@ radial_status launch_fwd(const radial_csr* c, const radial_desc* d, const void* 
   return RADIAL_OK;
 }
 
+template <int D>
+radial_status launch_bwd(const radial_csr* c, const radial_desc* d, const void* dout, const void* q,
+                         const void* k, const void* v, const void* o, const float* lse, void* dq, void* dk,
+                         void* dv, float* dr, cudaStream_t st) {
+  const int64_t rows = static_cast<int64_t>(d->batch) * d->heads * d->n_tokens;
+  {
+    const int threads = 256;
+    const int64_t blocks = (rows * 16 + threads - 1) / threads;
+    bwd_rowdot_kernel<D><<<static_cast<unsigned>(blocks), threads, 0, st>>>(
+        reinterpret_cast<const __nv_bfloat16*>(dout), reinterpret_cast<const __nv_bfloat16*>(o), d->heads,
+        d->n_tokens, d->stride_b, d->stride_h, d->stride_n, rows, dr);
+    RADIAL_LAUNCHED();
+  }
+  CUtensorMap mq, mk, mv, mdo;
+  radial_status rs;
+  if ((rs = make_bhnd_map(&mq, q, *d)) != RADIAL_OK) return rs;
+  if ((rs = make_bhnd_map(&mk, k, *d)) != RADIAL_OK) return rs;
+  if ((rs = make_bhnd_map(&mv, v, *d)) != RADIAL_OK) return rs;
+  if ((rs = make_bhnd_map(&mdo, dout, *d)) != RADIAL_OK) return rs;
+  BwdParams p;
+  p.row_ptr = c->plan.row_ptr;
+  p.col_idx = c->plan.col_idx;
+  p.kind = c->plan.kind;
+  p.row_order = c->plan.row_order;
+  p.col_ptr = c->plan.col_ptr;
+  p.row_idx = c->plan.row_idx;
+  p.kind_t = c->plan.kind_t;
+  p.col_order = c->plan.col_order;
+  p.nt = c->plan.nb;
+  p.f = c->f;
+  p.s = c->s;
+  p.n = c->n;
+  p.sink = c->sink;
+  p.heads = d->heads;
+  p.items = d->batch * d->heads * c->plan.nb;
+  p.sb = d->stride_b;
+  p.sh = d->stride_h;
+  p.sn = d->stride_n;
+  p.lse = lse;
+  p.dr = dr;
+  p.dq = reinterpret_cast<__nv_bfloat16*>(dq);
+  p.dk = reinterpret_cast<__nv_bfloat16*>(dk);
+  p.dv = reinterpret_cast<__nv_bfloat16*>(dv);
+  p.scale = softmax_scale(d);
+  p.scale_log2 = p.scale * 1.4426950408889634f;
+  const int smem = BwdCfg<D>::SMEM_BYTES;
+  RADIAL_CUDA(cudaFuncSetAttribute(radial_bwd_dkdv_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
+  RADIAL_CUDA(cudaFuncSetAttribute(radial_bwd_dq_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
+  const int grid = p.items < sm_count() ? p.items : sm_count();
+  radial_bwd_dkdv_kernel<D><<<grid, 192, smem, st>>>(mq, mk, mv, mdo, p);
+  RADIAL_LAUNCHED();
+  radial_bwd_dq_kernel<D><<<grid, 192, smem, st>>>(mq, mk, mv, mdo, p);
+  RADIAL_LAUNCHED();
+  return RADIAL_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -396,9 +471,7 @@ radial_status radial_attn_fwd(const radial_csr* c, const radial_desc* d, const v
 size_t radial_attn_bwd_workspace_size(const radial_desc* d) {
   if (!d || d->batch < 1 || d->heads < 1 || d->n_tokens < 1 || d->head_dim < 1) return 0;
   const size_t rows = static_cast<size_t>(d->batch) * d->heads * d->n_tokens;
-  const size_t dq = rows * d->head_dim * sizeof(float);
-  const size_t dr = rows * sizeof(float);
-  return ((dq + 255) & ~size_t(255)) + ((dr + 255) & ~size_t(255));
+  return (rows * sizeof(float) + 255) & ~size_t(255);
 }
 
 radial_status radial_attn_bwd(const radial_csr* c, const radial_desc* d, const void* dout, const void* q,
@@ -406,9 +479,21 @@ radial_status radial_attn_bwd(const radial_csr* c, const radial_desc* d, const v
                               void* dk, void* dv, void* workspace, size_t workspace_bytes, void* stream) {
   radial_status rs = check_desc(c, d);
   if (rs != RADIAL_OK) return rs;
-  (void)dout; (void)q; (void)k; (void)v; (void)o; (void)lse; (void)dq; (void)dk; (void)dv;
-  (void)workspace; (void)workspace_bytes; (void)stream;
-  return fail(RADIAL_EUNSUPPORTED, "backward not built yet");
+  if (!dout || !q || !k || !v || !o || !lse || !dq || !dk || !dv || !workspace)
+    return fail(RADIAL_EINVAL, "NULL tensor or workspace pointer");
+  if (!aligned16(dout) || !aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) ||
+      !aligned16(lse) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
+    return fail(RADIAL_EINVAL, "tensor pointers must be 16-byte aligned");
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+    return fail(RADIAL_EINVAL, "workspace must be 256-byte aligned");
+  if (workspace_bytes < radial_attn_bwd_workspace_size(d))
+    return fail(RADIAL_EINVAL, "workspace of %zu bytes is below the %zu required", workspace_bytes,
+                radial_attn_bwd_workspace_size(d));
+  if (d->head_dim == 128)
+    return launch_bwd<128>(c, d, dout, q, k, v, o, lse, dq, dk, dv, static_cast<float*>(workspace),
+                           as_stream(stream));
+  return launch_bwd<64>(c, d, dout, q, k, v, o, lse, dq, dk, dv, static_cast<float*>(workspace),
+                        as_stream(stream));
 }
 
 radial_status radial_device_status(void* stream) {
@@ -421,6 +506,22 @@ radial_status radial_device_status(void* stream) {
     return fail(RADIAL_EDEVICE, "a kernel aborted after a bounded wait ran out (code %d)", flag);
   }
   RADIAL_CUDA(cudaGetLastError());
+  return RADIAL_OK;
+}
+
+radial_status radial_selftest_bounded_wait(uint32_t limit_ms, void* stream) {
+  if (limit_ms < 1 || limit_ms > 2000) return fail(RADIAL_EINVAL, "limit_ms must be in [1, 2000]");
+  int* flag = nullptr;
+  RADIAL_CUDA(cudaMalloc(&flag, sizeof(int)));
+  selftest_bounded_wait_kernel<<<1, 32, 0, as_stream(stream)>>>(static_cast<uint64_t>(limit_ms) * 1000000ull, flag);
+  g_launches.fetch_add(1);
+  cudaError_t e = cudaGetLastError();
+  int h = 0;
+  if (e == cudaSuccess) e = cudaMemcpyAsync(&h, flag, sizeof(int), cudaMemcpyDeviceToHost, as_stream(stream));
+  if (e == cudaSuccess) e = cudaStreamSynchronize(as_stream(stream));
+  cudaFree(flag);
+  if (e != cudaSuccess) return fail(RADIAL_ECUDA, "self-test: %s", cudaGetErrorString(e));
+  if (h != 1) return fail(RADIAL_ECUDA, "self-test: the wait did not time out");
   return RADIAL_OK;
 }
 

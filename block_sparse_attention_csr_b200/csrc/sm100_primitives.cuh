@@ -75,25 +75,30 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 }
 
 // Wait until the phase with the given parity has completed.  Bounded: after
-// kWaitLimitNs the wait gives up, records the timeout in g_device_error and
-// in *abort (shared, seen by every warp of the CTA), and returns false.  Once
+// limit_ns the wait gives up, records the timeout in g_device_error and in
+// *abort (shared, seen by every warp of the CTA), and returns false.  Once
 // *abort is set every later wait returns false at once, so a CTA whose
 // protocol broke drains in bounded time instead of hanging.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
+__device__ __forceinline__ bool mbar_wait_limit(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                                uint64_t limit_ns) {
   if (mbar_try_wait(bar, parity)) return true;
-  uint64_t t0 = globaltimer_ns();
+  const uint64_t t0 = globaltimer_ns();
   uint32_t spins = 0;
   while (true) {
     if (*abort) return false;
     if (mbar_try_wait(bar, parity)) return true;
     if ((++spins & 63u) == 0u) {
-      if (globaltimer_ns() - t0 > kWaitLimitNs) {
+      if (globaltimer_ns() - t0 > limit_ns) {
         *abort = 1;
         atomicExch(&g_device_error, kErrWaitTimeout);
         return false;
       }
     }
   }
+}
+
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
+  return mbar_wait_limit(bar, parity, abort, kWaitLimitNs);
 }
 
 // Drain wait used on the way out of a kernel: ignores the abort flag (the

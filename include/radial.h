@@ -92,7 +92,7 @@ typedef struct radial_csr_info_t {
  * its active query blocks ascending; row_order / col_order list blocks by
  * active-tile count descending, ties by index ascending.
  * Runs on the device on `stream` and SYNCHRONISES it (the tile count sizes the
- * allocation).  Constraints: f >= 1, s >= 1, f*s < 2^31, B in {64, 128},
+ * allocation).  Constraints: f >= 1, s >= 1, f*s <= 2^30, B in {64, 128},
  * ceil(n/B) <= 32768.  On success *out owns device memory until
  * radial_csr_free.  Errors: RADIAL_EINVAL (bad sizes, null out/params,
  * non-zero reserved), RADIAL_EUNSUPPORTED (non-default central_band or
@@ -148,8 +148,9 @@ typedef struct radial_desc {
 radial_status radial_attn_fwd(const radial_csr* csr, const radial_desc* desc, const void* q,
                               const void* k, const void* v, void* o, float* lse, void* stream);
 
-/* Bytes of device workspace radial_attn_bwd needs for this shape (fp32 dQ
- * accumulator plus per-row dO.O sums).  Host only. */
+/* Bytes of device workspace radial_attn_bwd needs for this shape: one fp32
+ * per (batch, head, token) for the row sums rowsum(dO o O), rounded up to
+ * 256 bytes.  Returns 0 for a NULL or empty desc.  Host only. */
 size_t radial_attn_bwd_workspace_size(const radial_desc* desc);
 
 /* Backward of Eq.2 under the mask (the gradients LoRA fine-tuning, §4.3,
@@ -167,6 +168,14 @@ radial_status radial_attn_bwd(const radial_csr* csr, const radial_desc* desc, co
  * on a bounded wait since the last call (RADIAL_EDEVICE, then cleared), or a
  * CUDA error is pending (RADIAL_ECUDA).  RADIAL_OK otherwise. */
 radial_status radial_device_status(void* stream);
+
+/* Failure-detection self-test: launches one warp that waits on an mbarrier
+ * nothing completes, with a wait limit of limit_ms (1..2000) milliseconds.
+ * The bounded wait gives up, the kernel returns normally and records the
+ * abort, so a following radial_device_status() reports RADIAL_EDEVICE and
+ * the context stays usable.  Synchronous.  RADIAL_OK if the wait timed out
+ * as designed. */
+radial_status radial_selftest_bounded_wait(uint32_t limit_ms, void* stream);
 
 /* Static text for a status code. */
 const char* radial_status_str(radial_status s);

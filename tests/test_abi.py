@@ -88,7 +88,7 @@ def test_bwd_workspace_size(lib):
     d = B.radial_desc()
     d.batch, d.heads, d.n_tokens, d.head_dim = 1, 2, 1000, 128
     ws = lib.radial_attn_bwd_workspace_size(ctypes.byref(d))
-    assert ws >= 2 * 1000 * 128 * 4 + 2 * 1000 * 4
+    assert ws >= 2 * 1000 * 4          # one fp32 row sum per (head, token)
     assert ws % 256 == 0
     d.heads = 0
     assert lib.radial_attn_bwd_workspace_size(ctypes.byref(d)) == 0
