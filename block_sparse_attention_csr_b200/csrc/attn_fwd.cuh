@@ -126,7 +126,12 @@ __device__ __forceinline__ void row_mask_bits(const FwdParams& p, int i, int k, 
   }
 }
 
-template <int D>
+// kFastSoftmax: tree reductions, packed fp32x2 FMA / add, and every
+// kPolyEvery-th pair of exponentials on the FMA pipe (exp2_poly_x2) to take
+// load off the MUFU pipe; otherwise the plain one-MUFU-per-element loop.
+constexpr int kPolyEvery = 4;
+
+template <int D, bool kFastSoftmax>
 __global__ void __launch_bounds__(192, 1)
     radial_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                       const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
@@ -310,9 +315,21 @@ __global__ void __launch_bounds__(192, 1)
           for (int c = 0; c < 128; ++c)
             if (!((mw[c >> 5] >> (c & 31)) & 1u)) sv[c] = -INFINITY;
         }
-        float tmax = sv[0];
+        float tmax;
+        if constexpr (kFastSoftmax) {
+          float acc[4] = {sv[0], sv[1], sv[2], sv[3]};
 #pragma unroll
-        for (int c = 1; c < 128; ++c) tmax = fmaxf(tmax, sv[c]);
+          for (int c = 4; c + 8 <= 128; c += 8)
+#pragma unroll
+            for (int k = 0; k < 4; ++k) acc[k] = max3f(acc[k], sv[c + k], sv[c + 4 + k]);
+#pragma unroll
+          for (int k = 0; k < 4; ++k) acc[k] = fmaxf(acc[k], sv[124 + k]);
+          tmax = max3f(acc[0], acc[1], fmaxf(acc[2], acc[3]));
+        } else {
+          tmax = sv[0];
+#pragma unroll
+          for (int c = 1; c < 128; ++c) tmax = fmaxf(tmax, sv[c]);
+        }
         const float m_tile = tmax * p.scale_log2;  // -inf stays -inf (scale > 0)
         const bool grow = m_tile > m + kRescaleThreshold;
         if (j > 0) {
@@ -347,17 +364,49 @@ __global__ void __launch_bounds__(192, 1)
         }
         const float m_use = (m == -INFINITY) ? 0.f : m;
         float lsum = 0.f;
+        if constexpr (kFastSoftmax) {
+          const uint64_t sl2 = f2_pack(p.scale_log2, p.scale_log2);
+          const uint64_t negm = f2_pack(-m_use, -m_use);
+          uint64_t acc2[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll
-        for (int c = 0; c < 2; ++c) {
-          uint32_t w[32];
+          for (int c = 0; c < 2; ++c) {
+            uint32_t w[32];
 #pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            const float x0 = ex2_approx(fmaf(sv[c * 64 + 2 * e], p.scale_log2, -m_use));
-            const float x1 = ex2_approx(fmaf(sv[c * 64 + 2 * e + 1], p.scale_log2, -m_use));
-            lsum += x0 + x1;
-            w[e] = pack_bf16x2(x0, x1);
+            for (int e = 0; e < 32; ++e) {
+              const int i0 = c * 64 + 2 * e;
+              const uint64_t x = f2_fma(f2_pack(sv[i0], sv[i0 + 1]), sl2, negm);
+              uint64_t pe;
+              if ((e % kPolyEvery) == kPolyEvery - 1) {
+                pe = exp2_poly_x2(x);
+              } else {
+                float x0, x1;
+                f2_unpack(x, x0, x1);
+                pe = f2_pack(ex2_approx(x0), ex2_approx(x1));
+              }
+              acc2[e & 3] = f2_add(acc2[e & 3], pe);
+              float p0, p1;
+              f2_unpack(pe, p0, p1);
+              w[e] = pack_bf16x2(p0, p1);
+            }
+            tmem_st32(tmem + lane_addr + C::TM_P0 + sb * 64 + c * 32, w);
           }
-          tmem_st32(tmem + lane_addr + C::TM_P0 + sb * 64 + c * 32, w);
+          const uint64_t s01 = f2_add(f2_add(acc2[0], acc2[1]), f2_add(acc2[2], acc2[3]));
+          float s0, s1;
+          f2_unpack(s01, s0, s1);
+          lsum = s0 + s1;
+        } else {
+#pragma unroll
+          for (int c = 0; c < 2; ++c) {
+            uint32_t w[32];
+#pragma unroll
+            for (int e = 0; e < 32; ++e) {
+              const float x0 = ex2_approx(fmaf(sv[c * 64 + 2 * e], p.scale_log2, -m_use));
+              const float x1 = ex2_approx(fmaf(sv[c * 64 + 2 * e + 1], p.scale_log2, -m_use));
+              lsum += x0 + x1;
+              w[e] = pack_bf16x2(x0, x1);
+            }
+            tmem_st32(tmem + lane_addr + C::TM_P0 + sb * 64 + c * 32, w);
+          }
         }
         l += lsum;
         tmem_wait_st();

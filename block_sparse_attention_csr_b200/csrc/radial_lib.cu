@@ -11,6 +11,7 @@
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
+#include <cstdlib>
 #include <cstring>
 #include <mutex>
 #include <string>
@@ -39,6 +40,18 @@ __global__ void selftest_bounded_wait_kernel(uint64_t limit_ns, int* waited_out)
   const bool ok = mbar_wait_limit(&bar, 0, &abort_s, limit_ns);
   __syncwarp();
   if (threadIdx.x == 0) *waited_out = ok ? 0 : 1;
+}
+
+// Evaluates exp2_poly_x2 (the FMA-pipe exponential of the forward softmax)
+// on n inputs, for testing it against its error bound.
+__global__ void selftest_exp2_kernel(const float* __restrict__ x, float* __restrict__ y, int n) {
+  const int i = 2 * (blockIdx.x * blockDim.x + threadIdx.x);
+  if (i >= n) return;
+  const float a = x[i], b = (i + 1 < n) ? x[i + 1] : 0.f;
+  float r0, r1;
+  f2_unpack(exp2_poly_x2(f2_pack(a, b)), r0, r1);
+  y[i] = r0;
+  if (i + 1 < n) y[i + 1] = r1;
 }
 }  // namespace radial
 
@@ -359,6 +372,16 @@ radial_status check_desc(const radial_csr* c, const radial_desc* d) {
   return RADIAL_OK;
 }
 
+// RADIAL_FWD_SOFTMAX=classic selects the one-MUFU-per-element softmax loop
+// (kept for comparison); the default is the packed / partly polynomial one.
+bool fwd_classic_softmax() {
+  static const bool classic = [] {
+    const char* e = std::getenv("RADIAL_FWD_SOFTMAX");
+    return e && std::strcmp(e, "classic") == 0;
+  }();
+  return classic;
+}
+
 float softmax_scale(const radial_desc* d) {
   return d->scale > 0.f ? d->scale : 1.0f / std::sqrt(static_cast<float>(d->head_dim));
 }
@@ -390,9 +413,14 @@ radial_status launch_fwd(const radial_csr* c, const radial_desc* d, const void* 
   p.lse = lse;
   p.scale_log2 = softmax_scale(d) * 1.4426950408889634f;
   const int smem = FwdCfg<D>::SMEM_BYTES;
-  RADIAL_CUDA(cudaFuncSetAttribute(radial_fwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
   const int grid = p.items < sm_count() ? p.items : sm_count();
-  radial_fwd_kernel<D><<<grid, 192, smem, st>>>(mq, mk, mv, p);
+  if (fwd_classic_softmax()) {
+    RADIAL_CUDA(cudaFuncSetAttribute(radial_fwd_kernel<D, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
+    radial_fwd_kernel<D, false><<<grid, 192, smem, st>>>(mq, mk, mv, p);
+  } else {
+    RADIAL_CUDA(cudaFuncSetAttribute(radial_fwd_kernel<D, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
+    radial_fwd_kernel<D, true><<<grid, 192, smem, st>>>(mq, mk, mv, p);
+  }
   RADIAL_LAUNCHED();
   return RADIAL_OK;
 }
@@ -522,6 +550,15 @@ radial_status radial_selftest_bounded_wait(uint32_t limit_ms, void* stream) {
   cudaFree(flag);
   if (e != cudaSuccess) return fail(RADIAL_ECUDA, "self-test: %s", cudaGetErrorString(e));
   if (h != 1) return fail(RADIAL_ECUDA, "self-test: the wait did not time out");
+  return RADIAL_OK;
+}
+
+radial_status radial_selftest_exp2(const float* x, float* y, int32_t n, void* stream) {
+  if (!x || !y || n < 1) return fail(RADIAL_EINVAL, "bad arguments");
+  const int threads = 256;
+  const int blocks = ((n + 1) / 2 + threads - 1) / threads;
+  selftest_exp2_kernel<<<blocks, threads, 0, as_stream(stream)>>>(x, y, n);
+  RADIAL_LAUNCHED();
   return RADIAL_OK;
 }
 

@@ -127,20 +127,38 @@ def token_mask(f, s, sink=True):
     return allowed_tokens(a[:, None], a[None, :], s, sink)
 
 
+def _mask_from_table(qi, qk, kj, kl, f, s, sink):
+    """allowed() over a (queries x keys) grid using the per-distance table
+    (h(d), c(d)) of distance_table() instead of recomputing it per pair.
+    Same predicate, int32 arithmetic."""
+    H, Cp = distance_table(f, s)
+    H = H.astype(np.int32)
+    Cp = Cp.astype(np.int32)
+    d = np.abs(qi[:, None] - kj[None, :])
+    h = H[d]
+    out = np.abs(qk[:, None] - kl[None, :]) <= h          # h < 0 never passes
+    if (H < 0).any():
+        c = Cp[d]
+        out |= (h < 0) & (d % c == 0) & (qk[:, None] == kl[None, :])
+    if sink:
+        out |= (kj == 0)[None, :]
+    return out
+
+
 def row_mask(rows, f, s, sink=True):
     """Boolean mask of the given query rows against all n keys."""
     n = f * s
-    b = np.arange(n, dtype=np.int64)
-    rows = np.asarray(rows, dtype=np.int64)
-    return allowed_tokens(rows[:, None], b[None, :], s, sink)
+    rows = np.asarray(rows, dtype=np.int32)
+    b = np.arange(n, dtype=np.int32)
+    return _mask_from_table(rows // s, rows % s, b // s, b % s, f, s, sink)
 
 
 def col_mask(cols, f, s, sink=True):
     """Boolean mask of all n queries against the given key columns (n x len)."""
     n = f * s
-    a = np.arange(n, dtype=np.int64)
-    cols = np.asarray(cols, dtype=np.int64)
-    return allowed_tokens(a[:, None], cols[None, :], s, sink)
+    cols = np.asarray(cols, dtype=np.int32)
+    a = np.arange(n, dtype=np.int32)
+    return _mask_from_table(a // s, a % s, cols // s, cols % s, f, s, sink)
 
 
 # ---------------------------------------------------------------------------

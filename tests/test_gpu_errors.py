@@ -59,3 +59,17 @@ def test_bounded_wait_times_out_and_context_survives(setup):
     o, lse = rb.radial_attn_fwd(csr, q, k, v)      # the context still works
     rb.radial_device_status()
     assert torch.isfinite(o.float()).all()
+
+
+def test_polynomial_exp2_error_bound():
+    """The FMA-pipe exponential of the softmax: relative error below 1e-4 on
+    the range the softmax feeds it (x <= 8 after lazy rescaling), against fp64
+    2^x; clamped to a negligible positive value below -125."""
+    import numpy as np
+    x = torch.linspace(-124.0, 8.0, 2_000_001, device=DEV, dtype=torch.float32)
+    y = rb.radial_selftest_exp2(x)
+    ref = np.exp2(x.cpu().double().numpy())
+    rel = np.abs(y.cpu().double().numpy() - ref) / ref
+    assert rel.max() < 1e-4, rel.max()
+    z = rb.radial_selftest_exp2(torch.tensor([-float("inf"), -1000.0, -126.0], device=DEV))
+    assert (z.cpu() >= 0).all() and (z.cpu() < 1e-37).all()

@@ -248,3 +248,12 @@ def test_sampling_branch_reached_on_tiny_grid():
         ds = range(2 ** r, 2 ** (r + 1))
         kept = sum(int(m[0:s, d * s:(d + 1) * s].sum()) for d in ds)
         assert kept == sum(s for d in ds if d % int(M.sample_period(d, s)) == 0)
+
+
+@pytest.mark.parametrize("f,s,sink", [(8, 16, True), (64, 4, False), (64, 4, True), (9, 7, True), (1, 5, False)])
+def test_row_and_col_masks_equal_token_mask(f, s, sink):
+    full = M.token_mask(f, s, sink)
+    n = f * s
+    rows = np.arange(0, n, 3)
+    np.testing.assert_array_equal(M.row_mask(rows, f, s, sink), full[rows])
+    np.testing.assert_array_equal(M.col_mask(rows, f, s, sink), full[:, rows])
