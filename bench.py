@@ -305,6 +305,9 @@ def run_ours(args, rank, world, local_rank):
                             "note": "10*B^2*d flops per tile (5 GEMMs); the kernels issue 7 (dQ pass recomputes S, dP)"}
             del dq, dk, dv, ws
 
+    if rank == 0 and args.sweep:
+        extra["sweep"] = run_sweep(args, dev, stream, peak)
+
     # ---- end to end through the public API with host buffers
     e2e = None
     if rank == 0 and not args.quick:
@@ -360,7 +363,8 @@ def run_ours(args, rank, world, local_rank):
             try:
                 with open(tp) as fh:
                     tj = json.load(fh)
-                if tj.get("workload") == wl.name and tj.get("kernel_sha") == kernel_sha():
+                if (tj.get("workload") == wl.name and tj.get("kernel_sha") == kernel_sha()
+                        and tj.get("kernel") == fwd_kernel_name()):
                     traffic = tj.get("dram_bytes_per_launch")
             except Exception:
                 traffic = None
@@ -371,7 +375,7 @@ def run_ours(args, rank, world, local_rank):
             "config": config_of(wl, nnz),
             "pct_of_tensor_peak": 100.0 * value / world / peak,
             "mask_build_ms": mask_ms,
-            "roofline": {"bound": "tensor", "kernel": "radial_fwd_kernel<128>", "achieved": fwd_tf, "peak": peak,
+            "roofline": {"bound": "tensor", "kernel": fwd_kernel_name(), "achieved": fwd_tf, "peak": peak,
                          "unit": "TFLOP/s", "frac": fwd_tf / peak, "peak_source": f"{peak_src} bf16 burst",
                          "frac_of_sustained": fwd_tf / peak_sus, "traffic": traffic,
                          "algorithmic_flops_per_launch": tile_flops(wl, nnz), "launch_ms": fwd_ms},
@@ -384,10 +388,57 @@ def run_ours(args, rank, world, local_rank):
         print(json.dumps(line), flush=True)
 
 
+def run_sweep(args, dev, stream, peak):
+    """Radial forward against dense at fixed 3600 tokens/frame over the frame
+    counts of the scaling sweep: active tiles vs n log2 n, ms, TFLOP/s, % of
+    peak and the speedup over dense attention of the same shape (same kernels,
+    all-ones mask)."""
+    import numpy as np
+    import torch
+    import block_sparse_attention_csr_b200 as rb
+    from block_sparse_attention_csr_b200 import inputs as I
+
+    def timed(csr, q, k, v, o, lse, reps):
+        rb.radial_attn_fwd(csr, q, k, v, o=o, lse=lse, stream=stream)
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(reps)]
+        for a, b in ev:
+            a.record(stream)
+            rb.radial_attn_fwd(csr, q, k, v, o=o, lse=lse, stream=stream)
+            b.record(stream)
+        torch.cuda.synchronize(dev)
+        return float(np.median([a.elapsed_time(b) for a, b in ev]))
+
+    out = []
+    for f in (8, 16, 33, 66, 132):
+        wl = I.WORKLOADS[f"sweep_f{f}"]
+        q, k, v = I.draw(wl, device=dev, backward=False)
+        o = torch.empty_like(q)
+        lse = torch.empty(q.shape[:3], dtype=torch.float32, device=dev)
+        csr = rb.radial_mask_build(wl.frames, wl.tokens_per_frame, wl.block, sink=1)
+        nnz = rb.radial_csr_info(csr)["nnz"]
+        ms = timed(csr, q, k, v, o, lse, 5)
+        dcsr = rb.radial_mask_build_dense(wl.n, wl.block)
+        dnnz = rb.radial_csr_info(dcsr)["nnz"]
+        dms = timed(dcsr, q, k, v, o, lse, 2)
+        tf = tile_flops(wl, nnz) / (ms * 1e-3) / 1e12
+        out.append({"frames": f, "n_tokens": wl.n, "active_tiles": int(nnz), "dense_tiles": int(dnnz),
+                    "tiles_per_nlog2n": nnz / (wl.n * math.log2(wl.n)), "ms": ms, "tflops": tf,
+                    "pct_of_peak": 100 * tf / peak, "dense_ms": dms,
+                    "dense_tflops": tile_flops(wl, dnnz) / (dms * 1e-3) / 1e12, "speedup_vs_dense": dms / ms})
+        del q, k, v, o, lse, csr, dcsr
+        torch.cuda.empty_cache()
+    return out
+
+
+def fwd_kernel_name():
+    single = os.environ.get("RADIAL_FWD_KERNEL") == "single"
+    return "radial_fwd_kernel<128,1>" if single else "radial_fwd_pair_kernel<128>"
+
+
 def kernel_sha():
     import hashlib
     h = hashlib.sha1()
-    for f in ("attn_fwd.cuh", "sm100_primitives.cuh", "mask_build.cuh"):
+    for f in ("attn_fwd.cuh", "attn_fwd_pair.cuh", "sm100_primitives.cuh", "mask_build.cuh", "radial_lib.cu"):
         with open(os.path.join(ROOT, "block_sparse_attention_csr_b200", "csrc", f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:12]
@@ -454,6 +505,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--ref-rows", type=int, default=512)
+    ap.add_argument("--sweep", action="store_true", help="add the frame-count scaling sweep (radial vs dense)")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         args.warmup = 3

@@ -233,4 +233,65 @@ __global__ void rank_by_count_kernel(const int32_t* __restrict__ ptr, int nb,
   if (q < nb) order[rank] = q;
 }
 
+// ---------------------------------------------------------------------------
+// Pair plan: query tiles (2p, 2p+1) processed together by one CTA walk the
+// ascending union of their two CSR rows.  Per union entry: the key tile and
+// flags (bit 0 / 1: tile 2p / 2p+1 has it; bit 2 / 3: that tile's entry is
+// PARTIAL).
+// ---------------------------------------------------------------------------
+constexpr uint8_t kPairIn0 = 1, kPairIn1 = 2, kPairPart0 = 4, kPairPart1 = 8;
+
+template <bool kFill>
+__device__ __forceinline__ int merge_pair(const int32_t* __restrict__ row_ptr, const int32_t* __restrict__ col_idx,
+                                          const uint8_t* __restrict__ kind, int nt, int p,
+                                          int32_t* __restrict__ out_col, uint8_t* __restrict__ out_flag) {
+  const int t0 = 2 * p, t1 = 2 * p + 1;
+  int a = row_ptr[t0], ae = row_ptr[t0 + 1];
+  int b = 0, be = 0;
+  if (t1 < nt) {
+    b = row_ptr[t1];
+    be = row_ptr[t1 + 1];
+  }
+  int n = 0;
+  while (a < ae || b < be) {
+    const int ca = a < ae ? col_idx[a] : 0x7fffffff;
+    const int cb = b < be ? col_idx[b] : 0x7fffffff;
+    uint8_t fl = 0;
+    int c;
+    if (ca <= cb) {
+      c = ca;
+      fl |= kPairIn0 | (kind[a] != kTileFull ? kPairPart0 : 0);
+      ++a;
+    } else {
+      c = cb;
+    }
+    if (cb == c) {
+      fl |= kPairIn1 | (kind[b] != kTileFull ? kPairPart1 : 0);
+      ++b;
+    }
+    if (kFill) {
+      out_col[n] = c;
+      out_flag[n] = fl;
+    }
+    ++n;
+  }
+  return n;
+}
+
+__global__ void pair_count_kernel(const int32_t* __restrict__ row_ptr, const int32_t* __restrict__ col_idx,
+                                  const uint8_t* __restrict__ kind, int nt, int np, int32_t* __restrict__ cnt) {
+  const int p = blockIdx.x * blockDim.x + threadIdx.x;
+  if (p >= np) return;
+  cnt[p] = merge_pair<false>(row_ptr, col_idx, kind, nt, p, nullptr, nullptr);
+}
+
+__global__ void pair_fill_kernel(const int32_t* __restrict__ row_ptr, const int32_t* __restrict__ col_idx,
+                                 const uint8_t* __restrict__ kind, int nt, int np,
+                                 const int32_t* __restrict__ pair_ptr, int32_t* __restrict__ pcol,
+                                 uint8_t* __restrict__ pflag) {
+  const int p = blockIdx.x * blockDim.x + threadIdx.x;
+  if (p >= np) return;
+  merge_pair<true>(row_ptr, col_idx, kind, nt, p, pcol + pair_ptr[p], pflag + pair_ptr[p]);
+}
+
 }  // namespace radial

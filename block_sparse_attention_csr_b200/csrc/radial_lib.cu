@@ -19,6 +19,7 @@
 #include "../../include/radial.h"
 #include "attn_bwd.cuh"
 #include "attn_fwd.cuh"
+#include "attn_fwd_pair.cuh"
 #include "mask_build.cuh"
 #include "sm100_primitives.cuh"
 
@@ -156,11 +157,24 @@ struct TileLists {
   }
 };
 
+// Union walk of neighbouring query-tile pairs (2p, 2p+1) of the plan.
+struct PairLists {
+  int32_t np = 0;
+  int64_t nu = 0;
+  int32_t *ptr = nullptr, *col = nullptr, *order = nullptr;
+  uint8_t* flag = nullptr;
+  void release() {
+    cudaFree(ptr); cudaFree(col); cudaFree(order); cudaFree(flag);
+    *this = PairLists();
+  }
+};
+
 struct radial_csr {
   int32_t f = 0, s = 0, n = 0, B = 0, sink = 0, dense = 0, device = 0;
   TileLists user;   // at the caller's block size
   TileLists plan;   // at the kernels' 128-token tile (aliases `user` when B == 128)
   bool plan_owned = false;
+  PairLists pairs;  // pairs of plan rows for the two-tile forward
 };
 
 namespace {
@@ -213,6 +227,32 @@ radial_status lists_from_states(const uint8_t* states, int32_t nb, TileLists& L,
   return RADIAL_OK;
 }
 
+radial_status pairs_from_plan(const TileLists& P, PairLists& Q, cudaStream_t st) {
+  Q.np = (P.nb + 1) / 2;
+  int32_t* cnt = nullptr;
+  RADIAL_CUDA(cudaMalloc(&cnt, sizeof(int32_t) * Q.np));
+  RADIAL_CUDA(cudaMalloc(&Q.ptr, sizeof(int32_t) * (Q.np + 1)));
+  RADIAL_CUDA(cudaMalloc(&Q.order, sizeof(int32_t) * Q.np));
+  const int t = 128, g = (Q.np + t - 1) / t;
+  pair_count_kernel<<<g, t, 0, st>>>(P.row_ptr, P.col_idx, P.kind, P.nb, Q.np, cnt);
+  RADIAL_LAUNCHED();
+  exclusive_scan_kernel<<<1, 1024, 0, st>>>(cnt, Q.np, Q.ptr);
+  RADIAL_LAUNCHED();
+  int32_t nu = 0;
+  RADIAL_CUDA(cudaMemcpyAsync(&nu, Q.ptr + Q.np, sizeof(int32_t), cudaMemcpyDeviceToHost, st));
+  RADIAL_CUDA(cudaStreamSynchronize(st));
+  Q.nu = nu;
+  RADIAL_CUDA(cudaMalloc(&Q.col, sizeof(int32_t) * (nu > 0 ? nu : 1)));
+  RADIAL_CUDA(cudaMalloc(&Q.flag, nu > 0 ? nu : 1));
+  pair_fill_kernel<<<g, t, 0, st>>>(P.row_ptr, P.col_idx, P.kind, P.nb, Q.np, Q.ptr, Q.col, Q.flag);
+  RADIAL_LAUNCHED();
+  rank_by_count_kernel<<<(Q.np + 255) / 256, 256, 256 * sizeof(int32_t), st>>>(Q.ptr, Q.np, Q.order);
+  RADIAL_LAUNCHED();
+  RADIAL_CUDA(cudaStreamSynchronize(st));
+  cudaFree(cnt);
+  return RADIAL_OK;
+}
+
 radial_status build_mask(int32_t f, int32_t s, int32_t B, int32_t sink, int32_t dense,
                          radial_csr** out, cudaStream_t st) {
   const int64_t n64 = static_cast<int64_t>(f) * s;
@@ -232,6 +272,7 @@ radial_status build_mask(int32_t f, int32_t s, int32_t B, int32_t sink, int32_t 
     cudaFree(states);
     cudaFree(states128);
     if (r != RADIAL_OK) {
+      c->pairs.release();
       if (c->plan_owned) c->plan.release();
       c->user.release();
       delete c;
@@ -262,6 +303,8 @@ radial_status build_mask(int32_t f, int32_t s, int32_t B, int32_t sink, int32_t 
     rs = lists_from_states(states128, nt, c->plan, st);
     if (rs != RADIAL_OK) return cleanup(rs);
   }
+  rs = pairs_from_plan(c->plan, c->pairs, st);
+  if (rs != RADIAL_OK) return cleanup(rs);
   *out = c;
   return cleanup(RADIAL_OK);
 }
@@ -342,6 +385,7 @@ radial_status radial_csr_copy_to_host(const radial_csr* c, int32_t* row_ptr, int
 void radial_csr_free(radial_csr* c) {
   if (!c) return;
   cudaDeviceSynchronize();
+  c->pairs.release();
   if (c->plan_owned) c->plan.release();
   c->user.release();
   delete c;
@@ -384,6 +428,51 @@ bool fwd_classic_softmax() {
 
 float softmax_scale(const radial_desc* d) {
   return d->scale > 0.f ? d->scale : 1.0f / std::sqrt(static_cast<float>(d->head_dim));
+}
+
+// RADIAL_FWD_KERNEL=single selects the one-query-tile forward kernel; the
+// default is the two-tile (pair) kernel.
+bool fwd_single_tile() {
+  static const bool single = [] {
+    const char* e = std::getenv("RADIAL_FWD_KERNEL");
+    return e && std::strcmp(e, "single") == 0;
+  }();
+  return single;
+}
+
+template <int D>
+radial_status launch_fwd_pair(const radial_csr* c, const radial_desc* d, const void* q, const void* k,
+                              const void* v, void* o, float* lse, cudaStream_t st) {
+  CUtensorMap mq, mk, mv;
+  radial_status rs;
+  if ((rs = make_bhnd_map(&mq, q, *d)) != RADIAL_OK) return rs;
+  if ((rs = make_bhnd_map(&mk, k, *d)) != RADIAL_OK) return rs;
+  if ((rs = make_bhnd_map(&mv, v, *d)) != RADIAL_OK) return rs;
+  FwdPairParams p;
+  p.pair_ptr = c->pairs.ptr;
+  p.pair_col = c->pairs.col;
+  p.pair_flag = c->pairs.flag;
+  p.pair_order = c->pairs.order;
+  p.np = c->pairs.np;
+  p.nt = c->plan.nb;
+  p.f = c->f;
+  p.s = c->s;
+  p.n = c->n;
+  p.sink = c->sink;
+  p.heads = d->heads;
+  p.items = d->batch * d->heads * c->pairs.np;
+  p.o_sb = d->stride_b;
+  p.o_sh = d->stride_h;
+  p.o_sn = d->stride_n;
+  p.o = reinterpret_cast<__nv_bfloat16*>(o);
+  p.lse = lse;
+  p.scale_log2 = softmax_scale(d) * 1.4426950408889634f;
+  const int smem = FwdPairCfg<D>::SMEM_BYTES;
+  const int grid = p.items < sm_count() ? p.items : sm_count();
+  RADIAL_CUDA(cudaFuncSetAttribute(radial_fwd_pair_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
+  radial_fwd_pair_kernel<D><<<grid, 384, smem, st>>>(mq, mk, mv, p);
+  RADIAL_LAUNCHED();
+  return RADIAL_OK;
 }
 
 template <int D>
@@ -492,6 +581,10 @@ radial_status radial_attn_fwd(const radial_csr* c, const radial_desc* d, const v
   if (!q || !k || !v || !o || !lse) return fail(RADIAL_EINVAL, "NULL tensor pointer");
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
     return fail(RADIAL_EINVAL, "tensor pointers must be 16-byte aligned");
+  if (!fwd_single_tile()) {
+    if (d->head_dim == 128) return launch_fwd_pair<128>(c, d, q, k, v, o, lse, as_stream(stream));
+    return launch_fwd_pair<64>(c, d, q, k, v, o, lse, as_stream(stream));
+  }
   if (d->head_dim == 128) return launch_fwd<128>(c, d, q, k, v, o, lse, as_stream(stream));
   return launch_fwd<64>(c, d, q, k, v, o, lse, as_stream(stream));
 }

@@ -59,9 +59,21 @@ def run(fn_name, tasks, workers=None):
     if workers == 1:
         _init_worker(threads)
         return [fn(t) for t in tasks]
-    env_pp = os.environ.get("PYTHONPATH", "")
+    # Spawned workers import NumPy (and size the BLAS thread pool) before any
+    # initializer runs, so the limits go into the environment they inherit.
+    saved = {k: os.environ.get(k) for k in ("PYTHONPATH", "OPENBLAS_NUM_THREADS", "OMP_NUM_THREADS")}
+    env_pp = saved["PYTHONPATH"] or ""
     if ROOT not in env_pp.split(os.pathsep):
         os.environ["PYTHONPATH"] = ROOT + (os.pathsep + env_pp if env_pp else "")
-    ctx = mp.get_context("spawn")
-    with ctx.Pool(workers, initializer=_init_worker, initargs=(threads,)) as pool:
-        return pool.map(fn, tasks, chunksize=1)
+    os.environ["OPENBLAS_NUM_THREADS"] = str(threads)
+    os.environ["OMP_NUM_THREADS"] = str(threads)
+    try:
+        ctx = mp.get_context("spawn")
+        with ctx.Pool(workers, initializer=_init_worker, initargs=(threads,)) as pool:
+            return pool.map(fn, tasks, chunksize=1)
+    finally:
+        for k, v in saved.items():
+            if v is None:
+                os.environ.pop(k, None)
+            else:
+                os.environ[k] = v
