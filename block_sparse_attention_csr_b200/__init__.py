@@ -13,6 +13,7 @@ from ._binding import (  # noqa: F401
     load,
     make_desc,
     radial_attn_bwd,
+    radial_attn_bwd_noalloc,
     radial_attn_bwd_workspace_size,
     radial_attn_fwd,
     radial_csr_copy_to_host,

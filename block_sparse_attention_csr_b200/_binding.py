@@ -28,7 +28,7 @@ EXPORTED = (
     "radial_csr_copy_to_host", "radial_csr_free", "radial_attn_fwd",
     "radial_attn_bwd_workspace_size", "radial_attn_bwd", "radial_device_status",
     "radial_status_str", "radial_last_error", "radial_launch_count", "radial_selftest_bounded_wait",
-    "radial_selftest_exp2",
+    "radial_selftest_exp2", "radial_attn_bwd_noalloc",
 )
 
 
@@ -92,6 +92,8 @@ def load(path=None):
         L.radial_attn_bwd_workspace_size.restype = sz
         L.radial_attn_bwd.argtypes = [vp, ctypes.POINTER(radial_desc)] + [vp] * 10 + [sz, vp]
         L.radial_attn_bwd.restype = ctypes.c_int
+        L.radial_attn_bwd_noalloc.argtypes = [vp, ctypes.POINTER(radial_desc)] + [vp] * 10
+        L.radial_attn_bwd_noalloc.restype = ctypes.c_int
         L.radial_device_status.argtypes = [vp]
         L.radial_device_status.restype = ctypes.c_int
         L.radial_status_str.argtypes = [ctypes.c_int]
@@ -252,6 +254,21 @@ def radial_attn_bwd(csr, do, q, k, v, o, lse, dq=None, dk=None, dv=None, workspa
                                   _ptr(o), _ptr(lse), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(workspace),
                                   ctypes.c_size_t(workspace.numel() * workspace.element_size()),
                                   _stream(stream)), "radial_attn_bwd")
+    return dq, dk, dv
+
+
+def radial_attn_bwd_noalloc(csr, do, q, k, v, o, lse, dq=None, dk=None, dv=None, scale=None, stream=None):
+    """Backward through the no-allocation entry point (no workspace; the library
+    uses its fixed device scratch).  Allocates the outputs (torch) when not given."""
+    import torch
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    _same_layout(q, k, v, o, do, dq, dk, dv)
+    desc = make_desc(q, scale)
+    _check(load().radial_attn_bwd_noalloc(csr.handle, ctypes.byref(desc), _ptr(do), _ptr(q), _ptr(k), _ptr(v),
+                                          _ptr(o), _ptr(lse), _ptr(dq), _ptr(dk), _ptr(dv), _stream(stream)),
+           "radial_attn_bwd_noalloc")
     return dq, dk, dv
 
 

@@ -617,6 +617,67 @@ radial_status radial_attn_bwd(const radial_csr* c, const radial_desc* d, const v
                         as_stream(stream));
 }
 
+}  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Backward without any allocation: the row-sum scratch lives in a fixed
+// device array of this module instead of a caller-provided workspace.
+// ---------------------------------------------------------------------------
+namespace {
+constexpr size_t kNoAllocMaxRows = size_t(1) << 22;  // 4,194,304 fp32 row sums = 16 MiB
+}  // namespace
+
+// Loaded with the module on every device that uses the library; held until exit.
+static __device__ __align__(256) float g_noalloc_rowsum[kNoAllocMaxRows];
+
+namespace {
+std::mutex g_noalloc_mu;
+float* g_noalloc_ptr[64] = {};
+
+// Device address of g_noalloc_rowsum on the current device, looked up once per
+// device (the host-side name of the array is not a device address).
+radial_status noalloc_scratch(float** out) {
+  int dev = 0;
+  RADIAL_CUDA(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= 64) return fail(RADIAL_EUNSUPPORTED, "device index %d beyond 63", dev);
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (!g_noalloc_ptr[dev]) {
+    void* addr = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&addr, g_noalloc_rowsum);
+    if (e != cudaSuccess || !addr)
+      return fail(RADIAL_ECUDA, "cudaGetSymbolAddress of the row-sum scratch: %s", cudaGetErrorString(e));
+    g_noalloc_ptr[dev] = static_cast<float*>(addr);
+  }
+  *out = g_noalloc_ptr[dev];
+  return RADIAL_OK;
+}
+}  // namespace
+
+extern "C" {
+
+radial_status radial_attn_bwd_noalloc(const radial_csr* c, const radial_desc* d, const void* dout,
+                                      const void* q, const void* k, const void* v, const void* o,
+                                      const float* lse, void* dq, void* dk, void* dv, void* stream) {
+  radial_status rs = check_desc(c, d);
+  if (rs != RADIAL_OK) return rs;
+  if (!dout || !q || !k || !v || !o || !lse || !dq || !dk || !dv)
+    return fail(RADIAL_EINVAL, "NULL tensor pointer");
+  if (!aligned16(dout) || !aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) ||
+      !aligned16(lse) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
+    return fail(RADIAL_EINVAL, "tensor pointers must be 16-byte aligned");
+  const size_t rows = static_cast<size_t>(d->batch) * d->heads * d->n_tokens;
+  if (rows > kNoAllocMaxRows)
+    return fail(RADIAL_EUNSUPPORTED,
+                "batch * heads * n_tokens = %zu exceeds the %zu rows of the fixed scratch of "
+                "radial_attn_bwd_noalloc; use radial_attn_bwd with a workspace",
+                rows, kNoAllocMaxRows);
+  float* scratch = nullptr;
+  if ((rs = noalloc_scratch(&scratch)) != RADIAL_OK) return rs;
+  if (d->head_dim == 128)
+    return launch_bwd<128>(c, d, dout, q, k, v, o, lse, dq, dk, dv, scratch, as_stream(stream));
+  return launch_bwd<64>(c, d, dout, q, k, v, o, lse, dq, dk, dv, scratch, as_stream(stream));
+}
+
 radial_status radial_device_status(void* stream) {
   RADIAL_CUDA(cudaStreamSynchronize(as_stream(stream)));
   int flag = 0;

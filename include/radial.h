@@ -164,6 +164,30 @@ radial_status radial_attn_bwd(const radial_csr* csr, const radial_desc* desc, co
                               const float* lse, void* dq, void* dk, void* dv, void* workspace,
                               size_t workspace_bytes, void* stream);
 
+/* Backward for callers that cannot allocate device memory: the same
+ * computation as radial_attn_bwd, with no workspace argument.  The paper has
+ * no counterpart to this call; it exists for callers that cannot hand the
+ * library a workspace: code running in a plugin or callback interface that
+ * gives it no allocator, processes whose device memory is entirely reserved by
+ * another framework's pool, and latency-critical loops that must not call
+ * cudaMalloc because it can synchronise the device.
+ * The per-row scratch (one fp32 per (batch, head, token)) is a fixed array in
+ * the library's device memory of 4,194,304 floats (16 MiB), which every GPU
+ * that loads the library holds until the process exits.  Calls with
+ * batch * heads * n_tokens above 4,194,304 return RADIAL_EUNSUPPORTED and launch
+ * nothing.  The call allocates nothing: no cudaMalloc, no cudaFree, no
+ * allocating library routine.  The first call on a device looks up the
+ * array's device address (cudaGetSymbolAddress, once per device, with that
+ * device current); make that first call before any stream capture.  Every
+ * call shares the one array per device, which keeps the last call's contents
+ * (each call overwrites every row it reads before reading it), so calls that
+ * overlap on the GPU, on different streams or threads, race and must be
+ * serialised by the caller.  Arguments, layout and errors otherwise as for
+ * radial_attn_bwd.  Asynchronous. */
+radial_status radial_attn_bwd_noalloc(const radial_csr* csr, const radial_desc* desc, const void* dout,
+                                      const void* q, const void* k, const void* v, const void* o,
+                                      const float* lse, void* dq, void* dk, void* dv, void* stream);
+
 /* Synchronise `stream` and report whether any kernel of this library aborted
  * on a bounded wait since the last call (RADIAL_EDEVICE, then cleared), or a
  * CUDA error is pending (RADIAL_ECUDA).  RADIAL_OK otherwise. */
