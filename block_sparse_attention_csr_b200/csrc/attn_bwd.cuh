@@ -154,10 +154,13 @@ __device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
 // ---------------------------------------------------------------------------
 // 2. dK, dV: key-major walk of the CSC
 // ---------------------------------------------------------------------------
-// TMEM: dK [0,D) dV [128,128+D) S^T [256,384) dP^T [384,512);
-// P^T (bf16) overwrites S^T columns [256,320), dS^T overwrites [384,448).
+// TMEM: dK [0,D) dV [128,128+D) S^T [256,384) dP^T [384,512).  Warps: 0
+// producer, 1 MMA, 2-3 idle, 4-7 and 8-11 the two elementwise warpgroups
+// (query columns [0,64) and [64,128) of each tile).  Warpgroup wg writes its
+// bf16 P^T over S^T columns [64 wg, 64 wg + 32) and its dS^T over dP^T columns
+// [64 wg, 64 wg + 32), i.e. over values it has already read.
 template <int D>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(384, 1)
     radial_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                            const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
                            const BwdParams p) {
@@ -178,12 +181,12 @@ __global__ void __launch_bounds__(192, 1)
     bars->abort = 0;
     mbar_init(&bars->fix_full, 1);
     mbar_init(&bars->fix_empty, 1);
-    mbar_init(&bars->acc_empty, 128);
+    mbar_init(&bars->acc_empty, 256);
     mbar_init(&bars->mma_done, 1);
     mbar_init(&bars->s_full, 1);
     mbar_init(&bars->s_free, 128);
     for (int b = 0; b < 2; ++b) {
-      mbar_init(&bars->ew_full[b], 128);
+      mbar_init(&bars->ew_full[b], 256);
       mbar_init(&bars->mma2_done[b], 1);
       mbar_init(&bars->st_full[b], 1);
       mbar_init(&bars->st_empty[b], 1);
@@ -204,7 +207,7 @@ __global__ void __launch_bounds__(192, 1)
       uint32_t it = 0, item_i = 0;
       for (int item = blockIdx.x; item < p.items; item += gridDim.x, ++item_i) {
         const int bh = item / p.nt;
-        const int u = p.col_order[item - bh * p.nt];
+        const int u = p.col_order ? p.col_order[item - bh * p.nt] : item - bh * p.nt;
         const int b = bh / p.heads, h = bh - b * p.heads;
         if (item_i > 0) mbar_wait(&bars->fix_empty, (item_i - 1) & 1, abort_flag);
         mbar_arrive_expect_tx(&bars->fix_full, 2 * C::TILE_BYTES);
@@ -238,7 +241,7 @@ __global__ void __launch_bounds__(192, 1)
       uint32_t it = 0, item_i = 0;
       for (int item = blockIdx.x; item < p.items; item += gridDim.x, ++item_i) {
         const int bh = item / p.nt;
-        const int u = p.col_order[item - bh * p.nt];
+        const int u = p.col_order ? p.col_order[item - bh * p.nt] : item - bh * p.nt;
         const uint32_t n_tiles = static_cast<uint32_t>(p.col_ptr[u + 1] - p.col_ptr[u]);
         mbar_wait(&bars->fix_full, item_i & 1, abort_flag);
         tc_fence_after();
@@ -268,12 +271,14 @@ __global__ void __launch_bounds__(192, 1)
           tc_fence_after();
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk) {  // K = 128 query rows, 16 per MMA
-            mma_ts(tmem + TM_DV, tmem + TM_S + kk * 8, smem_desc(ob + kk * 2048, 16384, 1024, kSwizzle128B),
+            mma_ts(tmem + TM_DV, tmem + TM_S + 64 * (kk >> 2) + 8 * (kk & 3),
+                   smem_desc(ob + kk * 2048, 16384, 1024, kSwizzle128B),
                    idesc_g, (j > 0 || kk > 0) ? 1u : 0u);
           }
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk) {
-            mma_ts(tmem + TM_DK, tmem + TM_DP + kk * 8, smem_desc(qb + kk * 2048, 16384, 1024, kSwizzle128B),
+            mma_ts(tmem + TM_DK, tmem + TM_DP + 64 * (kk >> 2) + 8 * (kk & 3),
+                   smem_desc(qb + kk * 2048, 16384, 1024, kSwizzle128B),
                    idesc_g, (j > 0 || kk > 0) ? 1u : 0u);
           }
           mma_commit(&bars->mma2_done[g & 1]);
@@ -285,16 +290,19 @@ __global__ void __launch_bounds__(192, 1)
       mma_commit(&bars->mma_done);
       mbar_wait_drain(&bars->mma_done, 0);
     }
-  } else {
+  } else if (warp >= 4) {
+    // Two warpgroups split each tile by query columns: warpgroup wg owns
+    // queries [64 wg, 64 wg + 64) of the tile, for all 128 key rows (lanes).
+    const int wg = (warp - 4) >> 2;
     const int quarter = warp & 3;
     const int row = quarter * 32 + lane;
-    const int tid = threadIdx.x - 64;  // 0..127 inside the warpgroup
     const uint32_t lane_addr = static_cast<uint32_t>(quarter * 32) << 16;
     constexpr float kLog2e = 1.4426950408889634f;
+    float* my_vec = sVec + wg * 256;  // [2 buffers][64 lse2 | 64 dr]
     uint32_t it = 0, item_i = 0;
     for (int item = blockIdx.x; item < p.items; item += gridDim.x, ++item_i) {
       const int bh = item / p.nt;
-      const int u = p.col_order[item - bh * p.nt];
+      const int u = p.col_order ? p.col_order[item - bh * p.nt] : item - bh * p.nt;
       const int b = bh / p.heads, h = bh - b * p.heads;
       const int key = u * 128 + row;
       const bool valid = key < p.n;
@@ -308,14 +316,16 @@ __global__ void __launch_bounds__(192, 1)
         const uint32_t g = it + j;
         const int t = p.row_idx[c0 + j];
         const bool partial = p.kind_t[c0 + j] != kTileFull;
-        // per-query statistics of this query tile -> shared memory
-        float* vbuf = sVec + (g & 1) * 256;
+        // this warpgroup's 64 queries: lse2 and dr -> shared memory
+        float* vbuf = my_vec + (g & 1) * 128;
         {
-          const int a = t * 128 + tid;
-          vbuf[tid] = a < p.n ? lse_bh[a] * kLog2e : INFINITY;
-          vbuf[128 + tid] = a < p.n ? dr_bh[a] : 0.f;
+          const int a = t * 128 + 64 * wg + (row & 63);
+          if (row < 64)
+            vbuf[row] = a < p.n ? lse_bh[a] * kLog2e : INFINITY;
+          else
+            vbuf[row] = a < p.n ? dr_bh[a] : 0.f;
         }
-        named_bar_sync(1, 128);
+        named_bar_sync(1 + wg, 128);
         uint32_t mw[4] = {0xffffffffu, 0xffffffffu, 0xffffffffu, 0xffffffffu};
         if (partial) {
           if (valid)
@@ -327,45 +337,47 @@ __global__ void __launch_bounds__(192, 1)
         __syncwarp();
         tc_fence_after();
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
+        for (int c = 0; c < 2; ++c) {
+          const int gc = 2 * wg + c;  // 32-column chunk of the tile
           uint32_t rs[32], rp[32];
-          tmem_ld32(tmem + lane_addr + TM_S + c * 32, rs);
-          tmem_ld32(tmem + lane_addr + TM_DP + c * 32, rp);
+          tmem_ld32(tmem + lane_addr + TM_S + gc * 32, rs);
+          tmem_ld32(tmem + lane_addr + TM_DP + gc * 32, rp);
           tmem_wait_ld();
+          const uint32_t bits = mw[gc];
           uint32_t pw[16], dw[16];
 #pragma unroll
           for (int e = 0; e < 16; ++e) {
             float pv[2], dv[2];
 #pragma unroll
             for (int z = 0; z < 2; ++z) {
-              const int qi = c * 32 + 2 * e + z;
-              const bool ok = (mw[qi >> 5] >> (qi & 31)) & 1u;
-              const float x = fmaf(__uint_as_float(rs[2 * e + z]), p.scale_log2, -vbuf[qi]);
+              const int ql = c * 32 + 2 * e + z;  // query index inside this warpgroup's 64
+              const bool ok = (bits >> (2 * e + z)) & 1u;
+              const float x = fmaf(__uint_as_float(rs[2 * e + z]), p.scale_log2, -vbuf[ql]);
               pv[z] = ok ? ex2_approx(x) : 0.f;
-              dv[z] = pv[z] * (__uint_as_float(rp[2 * e + z]) - vbuf[128 + qi]);
+              dv[z] = pv[z] * (__uint_as_float(rp[2 * e + z]) - vbuf[64 + ql]);
             }
             pw[e] = pack_bf16x2(pv[0], pv[1]);
             dw[e] = pack_bf16x2(dv[0], dv[1]);
           }
-          tmem_st16(tmem + lane_addr + TM_S + c * 16, pw);
-          tmem_st16(tmem + lane_addr + TM_DP + c * 16, dw);
+          // bf16 results go to this warpgroup's own columns, over data already read
+          tmem_st16(tmem + lane_addr + TM_S + 64 * wg + c * 16, pw);
+          tmem_st16(tmem + lane_addr + TM_DP + 64 * wg + c * 16, dw);
         }
         tmem_wait_st();
         tc_fence_before();
         mbar_arrive(&bars->ew_full[g & 1]);
       }
-      // epilogue: dK (scaled), dV
+      // epilogue: warpgroup 0 writes dK (scaled), warpgroup 1 writes dV
       const uint32_t g_last = it + n_tiles - 1;
       mbar_wait(&bars->mma2_done[g_last & 1], (g_last >> 1) & 1, abort_flag);
       __syncwarp();
       tc_fence_after();
       const int64_t off = static_cast<int64_t>(b) * p.sb + static_cast<int64_t>(h) * p.sh +
                           static_cast<int64_t>(valid ? key : 0) * p.sn;
-#pragma unroll
-      for (int which = 0; which < 2; ++which) {
-        const uint32_t col = which == 0 ? TM_DK : TM_DV;
-        const float mul = which == 0 ? p.scale : 1.0f;
-        __nv_bfloat16* dst = (which == 0 ? p.dk : p.dv) + off;
+      {
+        const uint32_t col = wg == 0 ? TM_DK : TM_DV;
+        const float mul = wg == 0 ? p.scale : 1.0f;
+        __nv_bfloat16* dst = (wg == 0 ? p.dk : p.dv) + off;
 #pragma unroll
         for (int c = 0; c < D / 32; ++c) {
           uint32_t r[32];
@@ -399,8 +411,10 @@ __global__ void __launch_bounds__(192, 1)
 // 3. dQ: query-major walk of the CSR
 // ---------------------------------------------------------------------------
 // TMEM: S [0,128) dP [128,256) dQ [256,256+D) dS0 [384,448) dS1 [448,512).
+// Warps: 0 producer, 1 MMA, 2-3 idle, 4-7 and 8-11 the elementwise
+// warpgroups (key columns [0,64) and [64,128) of each tile).
 template <int D>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(384, 1)
     radial_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                          const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
                          const BwdParams p) {
@@ -420,12 +434,12 @@ __global__ void __launch_bounds__(192, 1)
     bars->abort = 0;
     mbar_init(&bars->fix_full, 1);
     mbar_init(&bars->fix_empty, 1);
-    mbar_init(&bars->acc_empty, 128);
+    mbar_init(&bars->acc_empty, 256);
     mbar_init(&bars->mma_done, 1);
     mbar_init(&bars->s_full, 1);
-    mbar_init(&bars->s_free, 128);
+    mbar_init(&bars->s_free, 256);
     for (int b = 0; b < 2; ++b) {
-      mbar_init(&bars->ew_full[b], 128);
+      mbar_init(&bars->ew_full[b], 256);
       mbar_init(&bars->mma2_done[b], 1);
       mbar_init(&bars->st_full[b], 1);
       mbar_init(&bars->st_empty[b], 1);
@@ -446,7 +460,7 @@ __global__ void __launch_bounds__(192, 1)
       uint32_t it = 0, item_i = 0;
       for (int item = blockIdx.x; item < p.items; item += gridDim.x, ++item_i) {
         const int bh = item / p.nt;
-        const int t = p.row_order[item - bh * p.nt];
+        const int t = p.row_order ? p.row_order[item - bh * p.nt] : item - bh * p.nt;
         const int b = bh / p.heads, h = bh - b * p.heads;
         if (item_i > 0) mbar_wait(&bars->fix_empty, (item_i - 1) & 1, abort_flag);
         mbar_arrive_expect_tx(&bars->fix_full, 2 * C::TILE_BYTES);
@@ -493,7 +507,7 @@ __global__ void __launch_bounds__(192, 1)
       };
       for (int item = blockIdx.x; item < p.items; item += gridDim.x, ++item_i) {
         const int bh = item / p.nt;
-        const int t = p.row_order[item - bh * p.nt];
+        const int t = p.row_order ? p.row_order[item - bh * p.nt] : item - bh * p.nt;
         const uint32_t n_tiles = static_cast<uint32_t>(p.row_ptr[t + 1] - p.row_ptr[t]);
         mbar_wait(&bars->fix_full, item_i & 1, abort_flag);
         tc_fence_after();
@@ -525,7 +539,8 @@ __global__ void __launch_bounds__(192, 1)
       mma_commit(&bars->mma_done);
       mbar_wait_drain(&bars->mma_done, 0);
     }
-  } else {
+  } else if (warp >= 4) {
+    const int wg = (warp - 4) >> 2;  // key columns [64 wg, 64 wg + 64) of each tile
     const int quarter = warp & 3;
     const int row = quarter * 32 + lane;
     const uint32_t lane_addr = static_cast<uint32_t>(quarter * 32) << 16;
@@ -533,7 +548,7 @@ __global__ void __launch_bounds__(192, 1)
     uint32_t it = 0, item_i = 0;
     for (int item = blockIdx.x; item < p.items; item += gridDim.x, ++item_i) {
       const int bh = item / p.nt;
-      const int t = p.row_order[item - bh * p.nt];
+      const int t = p.row_order ? p.row_order[item - bh * p.nt] : item - bh * p.nt;
       const int b = bh / p.heads, h = bh - b * p.heads;
       const int a = t * 128 + row;
       const bool valid = a < p.n;
@@ -562,25 +577,26 @@ __global__ void __launch_bounds__(192, 1)
         __syncwarp();
         tc_fence_after();
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
+        for (int c = 0; c < 2; ++c) {
+          const int gc = 2 * wg + c;
           uint32_t rs[32], rp[32];
-          tmem_ld32(tmem + lane_addr + TM_S + c * 32, rs);
-          tmem_ld32(tmem + lane_addr + TM_DP + c * 32, rp);
+          tmem_ld32(tmem + lane_addr + TM_S + gc * 32, rs);
+          tmem_ld32(tmem + lane_addr + TM_DP + gc * 32, rp);
           tmem_wait_ld();
+          const uint32_t bits = mw[gc];
           uint32_t dw[16];
 #pragma unroll
           for (int e = 0; e < 16; ++e) {
             float dv[2];
 #pragma unroll
             for (int z = 0; z < 2; ++z) {
-              const int ci = c * 32 + 2 * e + z;
-              const bool ok = (mw[ci >> 5] >> (ci & 31)) & 1u;
+              const bool ok = (bits >> (2 * e + z)) & 1u;
               const float pv = ok ? ex2_approx(fmaf(__uint_as_float(rs[2 * e + z]), p.scale_log2, -lse2)) : 0.f;
               dv[z] = pv * (__uint_as_float(rp[2 * e + z]) - drow);
             }
             dw[e] = pack_bf16x2(dv[0], dv[1]);
           }
-          tmem_st16(tmem + lane_addr + TM_DS + db * 64 + c * 16, dw);
+          tmem_st16(tmem + lane_addr + TM_DS + db * 64 + gc * 16, dw);
         }
         tmem_wait_st();
         tc_fence_before();
@@ -594,16 +610,17 @@ __global__ void __launch_bounds__(192, 1)
       __nv_bfloat16* dst = p.dq + static_cast<int64_t>(b) * p.sb + static_cast<int64_t>(h) * p.sh +
                            static_cast<int64_t>(valid ? a : 0) * p.sn;
 #pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
+      for (int c = 0; c < D / 64; ++c) {
+        const int col = (D / 2) * wg + 32 * c;  // this warpgroup's half of the dQ row
         uint32_t r[32];
-        tmem_ld32(tmem + lane_addr + TM_DQ + c * 32, r);
+        tmem_ld32(tmem + lane_addr + TM_DQ + col, r);
         tmem_wait_ld();
         if (valid) {
           uint32_t pk[16];
 #pragma unroll
           for (int e = 0; e < 16; ++e)
             pk[e] = pack_bf16x2(__uint_as_float(r[2 * e]) * p.scale, __uint_as_float(r[2 * e + 1]) * p.scale);
-          uint4* o4 = reinterpret_cast<uint4*>(dst + c * 32);
+          uint4* o4 = reinterpret_cast<uint4*>(dst + col);
 #pragma unroll
           for (int v = 0; v < 4; ++v) o4[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
         }

@@ -44,7 +44,7 @@ struct FwdParams {
   const int32_t* row_ptr;
   const int32_t* col_idx;
   const uint8_t* kind;
-  const int32_t* order;  // query tiles, longest row first
+  const int32_t* order;  // query tiles, longest row first (nullptr: ascending)
   int32_t nt;            // query tiles per head
   // mask geometry for PARTIAL tiles
   int32_t f, s, n, sink;
@@ -185,7 +185,7 @@ __global__ void __launch_bounds__(192, 1)
       uint32_t it = 0, item_i = 0;
       for (int item = blockIdx.x; item < p.items; item += gridDim.x, ++item_i) {
         const int bh = item / p.nt;
-        const int t = p.order[item - bh * p.nt];
+        const int t = p.order ? p.order[item - bh * p.nt] : item - bh * p.nt;
         const int b = bh / p.heads, h = bh - b * p.heads;
         if (item_i > 0) mbar_wait(&bars->q_empty, (item_i - 1) & 1, abort_flag);
         mbar_arrive_expect_tx(&bars->q_full, C::TILE_BYTES);
@@ -242,7 +242,7 @@ __global__ void __launch_bounds__(192, 1)
       };
       for (int item = blockIdx.x; item < p.items; item += gridDim.x, ++item_i) {
         const int bh = item / p.nt;
-        const int t = p.order[item - bh * p.nt];
+        const int t = p.order ? p.order[item - bh * p.nt] : item - bh * p.nt;
         const uint32_t n_tiles = static_cast<uint32_t>(p.row_ptr[t + 1] - p.row_ptr[t]);
         mbar_wait(&bars->q_full, item_i & 1, abort_flag);
         tc_fence_after();
@@ -280,7 +280,7 @@ __global__ void __launch_bounds__(192, 1)
     uint32_t it = 0, item_i = 0;
     for (int item = blockIdx.x; item < p.items; item += gridDim.x, ++item_i) {
       const int bh = item / p.nt;
-      const int t = p.order[item - bh * p.nt];
+      const int t = p.order ? p.order[item - bh * p.nt] : item - bh * p.nt;
       const int b = bh / p.heads, h = bh - b * p.heads;
       const int a = t * 128 + row;
       const bool valid = a < p.n;

@@ -11,8 +11,8 @@
 // that tile alone.
 //
 // Warp roles (384 threads, 168 registers each):
-//   warp 0      TMA producer: Q0, Q1 once per item; K and V through two
-//               separate 2-slot rings, K running one union column ahead of V.
+//   warp 0      TMA producer: Q0, Q1 once per item; K and V through
+//               separate 3-slot / 2-slot rings, K one union column ahead of V.
 //   warps 2-3   idle (keep the softmax warps on warpgroup boundaries).
 //   warp 1      TMEM allocator, single-thread tcgen05.mma issuer.  Per union
 //               column u and tile i: first O_i += P_i(u') V(u') for the tile's
@@ -33,8 +33,12 @@
 // P_i(u') is consumed and O_i is up to date for a rescale.  S_i(u+1) is
 // issued after PV_i(u) in the same MMA stream and executes after it.
 //
-// Shared memory: Q0, Q1 + 2 K slots + 2 V slots, 128 x D bf16 each, 128-byte
-// swizzle in 64-column boxes.
+// Shared memory: Q0, Q1 + 3 K slots + 2 V slots, 128 x D bf16 each, 128-byte
+// swizzle in 64-column boxes (224 KB at D = 128).
+//
+// Work items are (batch*head, pair) in head-major order; within a head the
+// pairs run longest-first when an order array is given (the default), else in
+// ascending query position.
 #pragma once
 
 #include <cstdint>
@@ -65,17 +69,19 @@ template <int D>
 struct FwdPairCfg {
   static constexpr int TILE_BYTES = 128 * D * 2;
   static constexpr int NBOX = D / 64;
+  static constexpr int K_SLOTS = 3;
+  static constexpr int V_SLOTS = 2;
   static constexpr int SMEM_Q = 0;
   static constexpr int SMEM_K = 2 * TILE_BYTES;
-  static constexpr int SMEM_V = 4 * TILE_BYTES;
-  static constexpr int SMEM_BAR = 6 * TILE_BYTES;
+  static constexpr int SMEM_V = SMEM_K + K_SLOTS * TILE_BYTES;
+  static constexpr int SMEM_BAR = SMEM_V + V_SLOTS * TILE_BYTES;
   static constexpr int SMEM_BYTES = SMEM_BAR + 512 + 1024;
   static constexpr uint32_t TM_S = 0, TM_O = 256;
 };
 
 struct PairBars {
   uint64_t q_full, q_empty, mma_done;
-  uint64_t k_full[2], k_empty[2], v_full[2], v_empty[2];
+  uint64_t k_full[3], k_empty[3], v_full[2], v_empty[2];
   uint64_t s_full[2], p_full[2], o_full[2], o_empty[2];
   uint32_t tmem_base;
   int abort;
@@ -101,9 +107,11 @@ __global__ void __launch_bounds__(384, 1)
     mbar_init(&bars->q_full, 1);
     mbar_init(&bars->q_empty, 1);
     mbar_init(&bars->mma_done, 1);
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < C::K_SLOTS; ++i) {
       mbar_init(&bars->k_full[i], 1);
       mbar_init(&bars->k_empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
       mbar_init(&bars->v_full[i], 1);
       mbar_init(&bars->v_empty[i], 1);
       mbar_init(&bars->s_full[i], 1);
@@ -130,7 +138,7 @@ __global__ void __launch_bounds__(384, 1)
       tma_prefetch_desc(&tmV);
       uint32_t kc = 0, vc = 0, item_i = 0;
       auto load_k = [&](int kb, int h, int b) {
-        const uint32_t sl = kc & 1, use = kc >> 1;
+        const uint32_t sl = kc % C::K_SLOTS, use = kc / C::K_SLOTS;
         if (use > 0) mbar_wait(&bars->k_empty[sl], (use - 1) & 1, abort_flag);
         mbar_arrive_expect_tx(&bars->k_full[sl], C::TILE_BYTES);
 #pragma unroll
@@ -149,7 +157,7 @@ __global__ void __launch_bounds__(384, 1)
       };
       for (int item = blockIdx.x; item < p.items; item += gridDim.x, ++item_i) {
         const int bh = item / p.np;
-        const int pr = p.pair_order[item - bh * p.np];
+        const int pr = p.pair_order ? p.pair_order[item - bh * p.np] : item - bh * p.np;
         const int b = bh / p.heads, h = bh - b * p.heads;
         const bool two = 2 * pr + 1 < p.nt;
         if (item_i > 0) mbar_wait(&bars->q_empty, (item_i - 1) & 1, abort_flag);
@@ -166,7 +174,8 @@ __global__ void __launch_bounds__(384, 1)
           load_v(p.pair_col[u], h, b);
         }
       }
-      for (uint32_t x = (kc > 2 ? kc - 2 : 0); x < kc; ++x) mbar_wait_drain(&bars->k_full[x & 1], (x >> 1) & 1);
+      for (uint32_t x = (kc > C::K_SLOTS ? kc - C::K_SLOTS : 0); x < kc; ++x)
+        mbar_wait_drain(&bars->k_full[x % C::K_SLOTS], (x / C::K_SLOTS) & 1);
       for (uint32_t x = (vc > 2 ? vc - 2 : 0); x < vc; ++x) mbar_wait_drain(&bars->v_full[x & 1], (x >> 1) & 1);
     }
   } else if (warp == 1) {
@@ -180,7 +189,7 @@ __global__ void __launch_bounds__(384, 1)
       uint32_t icnt[2] = {0u, 0u};    // items completed per query tile
       for (int item = blockIdx.x; item < p.items; item += gridDim.x, ++item_i) {
         const int bh = item / p.np;
-        const int pr = p.pair_order[item - bh * p.np];
+        const int pr = p.pair_order ? p.pair_order[item - bh * p.np] : item - bh * p.np;
         const int u0 = p.pair_ptr[pr], u1 = p.pair_ptr[pr + 1];
         mbar_wait(&bars->q_full, item_i & 1, abort_flag);
         tc_fence_after();
@@ -204,10 +213,12 @@ __global__ void __launch_bounds__(384, 1)
           first_pv[i] = false;
           pending[i] = false;
         };
+        uint8_t fl_next = p.pair_flag[u0];
         for (int u = u0; u < u1; ++u) {
-          const uint8_t fl = p.pair_flag[u];
-          const uint32_t ks = kc & 1;
-          mbar_wait(&bars->k_full[ks], (kc >> 1) & 1, abort_flag);
+          const uint8_t fl = fl_next;
+          if (u + 1 < u1) fl_next = p.pair_flag[u + 1];
+          const uint32_t ks = kc % C::K_SLOTS;
+          mbar_wait(&bars->k_full[ks], (kc / C::K_SLOTS) & 1, abort_flag);
           tc_fence_after();
           const uint32_t kb = k_base + ks * C::TILE_BYTES;
 #pragma unroll
@@ -268,7 +279,7 @@ __global__ void __launch_bounds__(384, 1)
     uint32_t g = 0, icnt = 0;
     for (int item = blockIdx.x; item < p.items; item += gridDim.x) {
       const int bh = item / p.np;
-      const int pr = p.pair_order[item - bh * p.np];
+      const int pr = p.pair_order ? p.pair_order[item - bh * p.np] : item - bh * p.np;
       const int t = 2 * pr + ti;
       if (t >= p.nt) continue;  // odd tail: this pair has one tile
       const int b = bh / p.heads, h = bh - b * p.heads;
@@ -279,10 +290,16 @@ __global__ void __launch_bounds__(384, 1)
       const int u0 = p.pair_ptr[pr], u1 = p.pair_ptr[pr + 1];
       float m = -INFINITY, l = 0.f;
       bool first = true;
+      uint8_t fl_next = p.pair_flag[u0];
+      int kb_next = p.pair_col[u0];
       for (int u = u0; u < u1; ++u) {
-        const uint8_t fl = p.pair_flag[u];
+        const uint8_t fl = fl_next;
+        const int kb = kb_next;
+        if (u + 1 < u1) {
+          fl_next = p.pair_flag[u + 1];
+          kb_next = p.pair_col[u + 1];
+        }
         if (!(fl & in_bit)) continue;
-        const int kb = p.pair_col[u];
         mbar_wait(&bars->s_full[ti], g & 1, abort_flag);
         __syncwarp();
         tc_fence_after();
@@ -295,26 +312,29 @@ __global__ void __launch_bounds__(384, 1)
         }
         float sv[64];
         float acc[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+        // two TMEM round trips: chunks {0,1} (kept) then {2,3} (max only)
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          uint32_t r[32];
-          tmem_ld32(tm_s + c * 32, r);
+        for (int half = 0; half < 2; ++half) {
+          uint32_t r[64];
+          tmem_ld32(tm_s + half * 64, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
+          tmem_ld32(tm_s + half * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
           tmem_wait_ld();
-          float x[32];
+          float x[64];
           if (part) {
 #pragma unroll
-            for (int e = 0; e < 32; ++e) x[e] = ((mw[c] >> e) & 1u) ? __uint_as_float(r[e]) : -INFINITY;
+            for (int e = 0; e < 64; ++e)
+              x[e] = ((mw[2 * half + (e >> 5)] >> (e & 31)) & 1u) ? __uint_as_float(r[e]) : -INFINITY;
           } else {
 #pragma unroll
-            for (int e = 0; e < 32; ++e) x[e] = __uint_as_float(r[e]);
+            for (int e = 0; e < 64; ++e) x[e] = __uint_as_float(r[e]);
           }
 #pragma unroll
-          for (int e = 0; e < 32; e += 8)
+          for (int e = 0; e < 64; e += 8)
 #pragma unroll
             for (int k = 0; k < 4; ++k) acc[k] = max3f(acc[k], x[e + k], x[e + 4 + k]);
-          if (c < 2) {
+          if (half == 0) {
 #pragma unroll
-            for (int e = 0; e < 32; ++e) sv[c * 32 + e] = x[e];
+            for (int e = 0; e < 64; ++e) sv[e] = x[e];
           }
         }
         const float m_tile = max3f(acc[0], acc[1], fmaxf(acc[2], acc[3])) * p.scale_log2;
@@ -344,24 +364,8 @@ __global__ void __launch_bounds__(384, 1)
         const uint64_t sl2 = f2_pack(p.scale_log2, p.scale_log2);
         const uint64_t negm = f2_pack(-m_use, -m_use);
         uint64_t acc2[4] = {0ull, 0ull, 0ull, 0ull};
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          float x[32];
-          if (c < 2) {
-#pragma unroll
-            for (int e = 0; e < 32; ++e) x[e] = sv[c * 32 + e];
-          } else {
-            uint32_t r[32];
-            tmem_ld32(tm_s + c * 32, r);
-            tmem_wait_ld();
-            if (part) {
-#pragma unroll
-              for (int e = 0; e < 32; ++e) x[e] = ((mw[c] >> e) & 1u) ? __uint_as_float(r[e]) : -INFINITY;
-            } else {
-#pragma unroll
-              for (int e = 0; e < 32; ++e) x[e] = __uint_as_float(r[e]);
-            }
-          }
+        // P from 32 logits x -> 16 packed bf16 pairs into TMEM columns [16 c, 16 c + 16)
+        auto make_p = [&](const float (&x)[32], int c) {
           uint32_t w[16];
 #pragma unroll
           for (int e = 0; e < 16; ++e) {
@@ -380,6 +384,36 @@ __global__ void __launch_bounds__(384, 1)
             w[e] = pack_bf16x2(p0, p1);
           }
           tmem_st16(tm_s + c * 16, w);
+        };
+        {
+          float x0[32];
+#pragma unroll
+          for (int e = 0; e < 32; ++e) x0[e] = sv[e];
+          make_p(x0, 0);
+        }
+        // re-read chunk 2 while chunk 1 is turned into P (P only overwrites columns [0,64))
+        uint32_t r2[32], r3[32];
+        tmem_ld32(tm_s + 64, r2);
+        {
+          float x1[32];
+#pragma unroll
+          for (int e = 0; e < 32; ++e) x1[e] = sv[32 + e];
+          make_p(x1, 1);
+        }
+        tmem_ld32(tm_s + 96, r3);
+        tmem_wait_ld();
+#pragma unroll
+        for (int c = 2; c < 4; ++c) {
+          const uint32_t (&r)[32] = c == 2 ? r2 : r3;
+          float x[32];
+          if (part) {
+#pragma unroll
+            for (int e = 0; e < 32; ++e) x[e] = ((mw[c] >> e) & 1u) ? __uint_as_float(r[e]) : -INFINITY;
+          } else {
+#pragma unroll
+            for (int e = 0; e < 32; ++e) x[e] = __uint_as_float(r[e]);
+          }
+          make_p(x, c);
         }
         const uint64_t s01 = f2_add(f2_add(acc2[0], acc2[1]), f2_add(acc2[2], acc2[3]));
         float s0, s1;

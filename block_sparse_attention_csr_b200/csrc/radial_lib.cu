@@ -430,6 +430,18 @@ float softmax_scale(const radial_desc* d) {
   return d->scale > 0.f ? d->scale : 1.0f / std::sqrt(static_cast<float>(d->head_dim));
 }
 
+// Work-item order inside a head.  Default: longest row (column) first, which
+// measured best (it balances the tail of each launch).
+// RADIAL_SCHEDULE=natural: ascending tile position (the CTAs running at the
+// same time then share the K / V of a band of nearby frames).
+bool schedule_lpt() {
+  static const bool lpt = [] {
+    const char* e = std::getenv("RADIAL_SCHEDULE");
+    return !(e && std::strcmp(e, "natural") == 0);
+  }();
+  return lpt;
+}
+
 // RADIAL_FWD_KERNEL=single selects the one-query-tile forward kernel; the
 // default is the two-tile (pair) kernel.
 bool fwd_single_tile() {
@@ -452,7 +464,7 @@ radial_status launch_fwd_pair(const radial_csr* c, const radial_desc* d, const v
   p.pair_ptr = c->pairs.ptr;
   p.pair_col = c->pairs.col;
   p.pair_flag = c->pairs.flag;
-  p.pair_order = c->pairs.order;
+  p.pair_order = schedule_lpt() ? c->pairs.order : nullptr;
   p.np = c->pairs.np;
   p.nt = c->plan.nb;
   p.f = c->f;
@@ -487,7 +499,7 @@ radial_status launch_fwd(const radial_csr* c, const radial_desc* d, const void* 
   p.row_ptr = c->plan.row_ptr;
   p.col_idx = c->plan.col_idx;
   p.kind = c->plan.kind;
-  p.order = c->plan.row_order;
+  p.order = schedule_lpt() ? c->plan.row_order : nullptr;
   p.nt = c->plan.nb;
   p.f = c->f;
   p.s = c->s;
@@ -537,11 +549,11 @@ radial_status launch_bwd(const radial_csr* c, const radial_desc* d, const void* 
   p.row_ptr = c->plan.row_ptr;
   p.col_idx = c->plan.col_idx;
   p.kind = c->plan.kind;
-  p.row_order = c->plan.row_order;
+  p.row_order = schedule_lpt() ? c->plan.row_order : nullptr;
   p.col_ptr = c->plan.col_ptr;
   p.row_idx = c->plan.row_idx;
   p.kind_t = c->plan.kind_t;
-  p.col_order = c->plan.col_order;
+  p.col_order = schedule_lpt() ? c->plan.col_order : nullptr;
   p.nt = c->plan.nb;
   p.f = c->f;
   p.s = c->s;
@@ -563,9 +575,9 @@ radial_status launch_bwd(const radial_csr* c, const radial_desc* d, const void* 
   RADIAL_CUDA(cudaFuncSetAttribute(radial_bwd_dkdv_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
   RADIAL_CUDA(cudaFuncSetAttribute(radial_bwd_dq_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
   const int grid = p.items < sm_count() ? p.items : sm_count();
-  radial_bwd_dkdv_kernel<D><<<grid, 192, smem, st>>>(mq, mk, mv, mdo, p);
+  radial_bwd_dkdv_kernel<D><<<grid, 384, smem, st>>>(mq, mk, mv, mdo, p);
   RADIAL_LAUNCHED();
-  radial_bwd_dq_kernel<D><<<grid, 192, smem, st>>>(mq, mk, mv, mdo, p);
+  radial_bwd_dq_kernel<D><<<grid, 384, smem, st>>>(mq, mk, mv, mdo, p);
   RADIAL_LAUNCHED();
   return RADIAL_OK;
 }
