@@ -40,7 +40,8 @@ class RadialError(RuntimeError):
 
 class radial_params(ctypes.Structure):
     _fields_ = [("sink", ctypes.c_int32), ("central_band", ctypes.c_int32),
-                ("width_scale", ctypes.c_int32), ("reserved", ctypes.c_int32 * 5)]
+                ("width_scale_num", ctypes.c_int32), ("width_scale_den", ctypes.c_int32),
+                ("decay", ctypes.c_int32), ("reserved", ctypes.c_int32 * 3)]
 
 
 class radial_csr_info_t(ctypes.Structure):
@@ -156,10 +157,17 @@ def radial_params_default():
     return p
 
 
-def radial_mask_build(frames, tokens_per_frame, block, sink=1, central_band=1, width_scale=2,
-                      stream=None, reserved=None):
+DECAYS = {"radial": 0, "harmonic": 1}
+
+
+def radial_mask_build(frames, tokens_per_frame, block, sink=1, central_band=1, width_scale=(2, 1),
+                      decay="radial", stream=None, reserved=None):
+    """width_scale: (num, den) of the band-to-band width ratio; decay: "radial" or "harmonic"."""
     p = radial_params_default()
-    p.sink, p.central_band, p.width_scale = int(sink), int(central_band), int(width_scale)
+    num, den = (width_scale, 1) if isinstance(width_scale, int) else width_scale
+    p.sink, p.central_band = int(sink), int(central_band)
+    p.width_scale_num, p.width_scale_den = int(num), int(den)
+    p.decay = DECAYS[decay] if isinstance(decay, str) else int(decay)
     if reserved is not None:
         for i, r in enumerate(reserved):
             p.reserved[i] = int(r)

@@ -91,13 +91,14 @@ struct BwdParams {
   __nv_bfloat16* dv;
   float scale;
   float scale_log2;
+  const int32_t* hd;  // ablation-mask distance tables (nullptr: closed form)
+  const int32_t* cd;
 };
 
 // Allowed query rows (relative to a0, 128 wide) of key token b = j*s + l:
 // the transpose of row_mask_bits.
-__device__ __forceinline__ void col_mask_bits(int f_unused, int s, int n, int sink, int j, int l, int a0,
-                                              uint32_t (&mw)[4]) {
-  (void)f_unused;
+__device__ __forceinline__ void col_mask_bits(const int32_t* hd, const int32_t* cd, int s, int n, int sink,
+                                              int j, int l, int a0, uint32_t (&mw)[4]) {
   mw[0] = mw[1] = mw[2] = mw[3] = 0u;
   const int aend = min(a0 + 128, n);
   for (int i = a0 / s; i * s < aend; ++i) {
@@ -109,14 +110,13 @@ __device__ __forceinline__ void col_mask_bits(int f_unused, int s, int n, int si
       hi = seg_hi;
     } else {
       const int d = i > j ? i - j : j - i;
-      const int r = 31 - __clz(d > 1 ? d : 1);
-      const int h = (s >> r) - 1;
+      const int h = half_width_of(hd, s, d);
       const int center = i * s + l - a0;
       if (h >= 0) {
         lo = max(seg_lo, center - h);
         hi = min(seg_hi, center + h);
       } else {
-        const long long period = ((1LL << r) + s - 1) / s;
+        const long long period = period_of(cd, s, d);
         if (d % period != 0) continue;
         lo = max(seg_lo, center);
         hi = min(seg_hi, center);
@@ -329,7 +329,7 @@ __global__ void __launch_bounds__(384, 1)
         uint32_t mw[4] = {0xffffffffu, 0xffffffffu, 0xffffffffu, 0xffffffffu};
         if (partial) {
           if (valid)
-            col_mask_bits(p.f, p.s, p.n, p.sink, kj, kl, t * 128, mw);
+            col_mask_bits(p.hd, p.cd, p.s, p.n, p.sink, kj, kl, t * 128, mw);
           else
             mw[0] = mw[1] = mw[2] = mw[3] = 0u;
         }
@@ -565,8 +565,16 @@ __global__ void __launch_bounds__(384, 1)
         uint32_t mw[4] = {0xffffffffu, 0xffffffffu, 0xffffffffu, 0xffffffffu};
         if (partial) {
           mw[0] = mw[1] = mw[2] = mw[3] = 0u;
-          if (valid) row_mask_bits(FwdParams{nullptr, nullptr, nullptr, nullptr, 0, p.f, p.s, p.n, p.sink},
-                                   qi, qk, kb * 128, mw);
+          if (valid) {
+            FwdParams mp{};
+            mp.f = p.f;
+            mp.s = p.s;
+            mp.n = p.n;
+            mp.sink = p.sink;
+            mp.hd = p.hd;
+            mp.cd = p.cd;
+            row_mask_bits(mp, qi, qk, kb * 128, mw);
+          }
         }
         // dS buffer db was read by the dQ MMA of tile g-2
         if (g >= 2) {

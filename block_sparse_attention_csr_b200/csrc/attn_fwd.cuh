@@ -55,6 +55,9 @@ struct FwdParams {
   __nv_bfloat16* o;
   float* lse;
   float scale_log2;  // softmax scale * log2(e)
+  // ablation-mask distance tables (nullptr: the method's closed form)
+  const int32_t* hd;
+  const int32_t* cd;
 };
 
 template <int D>
@@ -109,14 +112,13 @@ __device__ __forceinline__ void row_mask_bits(const FwdParams& p, int i, int k, 
       hi = seg_hi;
     } else {
       const int d = i > j ? i - j : j - i;
-      const int r = 31 - __clz(d > 1 ? d : 1);
-      const int h = (p.s >> r) - 1;
+      const int h = half_width_of(p.hd, p.s, d);
       const int center = j * p.s + k - b0;
       if (h >= 0) {
         lo = max(seg_lo, center - h);
         hi = min(seg_hi, center + h);
       } else {
-        const long long period = ((1LL << r) + p.s - 1) / p.s;
+        const long long period = period_of(p.cd, p.s, d);
         if (d % period != 0) continue;
         lo = max(seg_lo, center);
         hi = min(seg_hi, center);

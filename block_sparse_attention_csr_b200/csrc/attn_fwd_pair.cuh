@@ -63,6 +63,8 @@ struct FwdPairParams {
   __nv_bfloat16* o;
   float* lse;
   float scale_log2;
+  const int32_t* hd;  // ablation-mask distance tables (nullptr: closed form)
+  const int32_t* cd;
 };
 
 template <int D>
@@ -276,6 +278,8 @@ __global__ void __launch_bounds__(384, 1)
     mp.s = p.s;
     mp.n = p.n;
     mp.sink = p.sink;
+    mp.hd = p.hd;
+    mp.cd = p.cd;
     uint32_t g = 0, icnt = 0;
     for (int item = blockIdx.x; item < p.items; item += gridDim.x) {
       const int bh = item / p.np;

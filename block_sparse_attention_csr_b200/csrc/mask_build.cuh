@@ -28,7 +28,24 @@ constexpr uint8_t kTilePartial = 2;
 
 struct MaskGeom {
   int32_t f, s, n, B, nb, sink;
+  // per-frame-distance half width h(d) and sampled-diagonal period c(d) of an
+  // ablation mask; nullptr selects the method's own closed form
+  const int32_t* hd;
+  const int32_t* cd;
 };
+
+// h(d) and c(d): the closed form r = floor(log2 max(d,1)), h = floor(s/2^r)-1,
+// c = ceil(2^r/s), or the table of an ablation mask.
+__device__ __forceinline__ int half_width_of(const int32_t* hd, int s, int d) {
+  if (hd) return hd[d];
+  const int r = 31 - __clz(d > 1 ? d : 1);
+  return (s >> r) - 1;
+}
+__device__ __forceinline__ long long period_of(const int32_t* cd, int s, int d) {
+  if (cd) return cd[d];
+  const int r = 31 - __clz(d > 1 ? d : 1);
+  return ((1LL << r) + s - 1) / s;
+}
 
 __device__ __forceinline__ int band_of(int d) {  // floor(log2(max(d,1)))
   return 31 - __clz(d > 1 ? d : 1);
@@ -44,8 +61,7 @@ __device__ __forceinline__ void segment_pair(const MaskGeom& g, int i, int k0, i
     return;
   }
   const int d = i > j ? i - j : j - i;
-  const int r = band_of(d);
-  const int h = (g.s >> r) - 1;
+  const int h = half_width_of(g.hd, g.s, d);
   int gap = l0 - k1;
   if (k0 - l1 > gap) gap = k0 - l1;
   if (gap < 0) gap = 0;
@@ -55,7 +71,7 @@ __device__ __forceinline__ void segment_pair(const MaskGeom& g, int i, int k0, i
     all = span <= h;
     return;
   }
-  const long long period = ((1LL << r) + g.s - 1) / g.s;
+  const long long period = period_of(g.cd, g.s, d);
   if (d % period == 0) {
     any = gap == 0;
     all = (k0 == k1) && (l0 == l1) && (k0 == l0);

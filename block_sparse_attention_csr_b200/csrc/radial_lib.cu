@@ -15,6 +15,7 @@
 #include <cstring>
 #include <mutex>
 #include <string>
+#include <vector>
 
 #include "../../include/radial.h"
 #include "attn_bwd.cuh"
@@ -171,6 +172,8 @@ struct PairLists {
 
 struct radial_csr {
   int32_t f = 0, s = 0, n = 0, B = 0, sink = 0, dense = 0, device = 0;
+  int32_t* hd = nullptr;  // ablation-mask half widths per frame distance (device; nullptr = method's rule)
+  int32_t* cd = nullptr;  // ablation-mask sampled-diagonal periods per frame distance
   TileLists user;   // at the caller's block size
   TileLists plan;   // at the kernels' 128-token tile (aliases `user` when B == 128)
   bool plan_owned = false;
@@ -253,7 +256,52 @@ radial_status pairs_from_plan(const TileLists& P, PairLists& Q, cudaStream_t st)
   return RADIAL_OK;
 }
 
-radial_status build_mask(int32_t f, int32_t s, int32_t B, int32_t sink, int32_t dense,
+// Ablation mask rule (see radial_params in radial.h).
+struct MaskRule {
+  int32_t central_band = 1, num = 2, den = 1, decay = 0;
+  bool is_default() const { return central_band == 1 && num == 2 * den && decay == 0; }
+};
+
+// h(d), c(d) for d in [0, f) in exact integer arithmetic (128-bit for the
+// band boundaries (cb+1) (num/den)^r).  false if the arithmetic would overflow.
+bool mask_rule_table(const MaskRule& m, int32_t f, int32_t s, std::vector<int32_t>& H, std::vector<int32_t>& C) {
+  typedef unsigned __int128 u128;
+  const u128 limit = static_cast<u128>(1) << 120;
+  H.assign(f, 0);
+  C.assign(f, 1);
+  int r = 1;
+  u128 P = static_cast<u128>(m.num), Q = static_cast<u128>(m.den);  // num^r, den^r
+  for (int32_t d = 0; d < f; ++d) {
+    int64_t w;
+    int64_t c = 1;
+    if (d <= m.central_band) {
+      w = s;
+    } else if (m.decay == 1) {
+      const int64_t e = static_cast<int64_t>(d) - m.central_band + 1;
+      w = s / e;
+      if (w < 1) c = (e + s - 1) / s;
+    } else {
+      // advance to the band with dist < (cb+1) sigma^r (bands only grow with d)
+      while (!(static_cast<u128>(d) * Q < static_cast<u128>(m.central_band + 1) * P)) {
+        P *= static_cast<u128>(m.num);
+        Q *= static_cast<u128>(m.den);
+        ++r;
+        if (P > limit || Q > limit) return false;
+      }
+      const u128 sQ = static_cast<u128>(s) * Q;
+      w = static_cast<int64_t>(sQ / P);
+      if (w < 1) {
+        const u128 cc = (P + sQ - 1) / sQ;
+        c = cc > static_cast<u128>(0x7fffffff) ? 0x7fffffff : static_cast<int64_t>(cc);
+      }
+    }
+    H[d] = static_cast<int32_t>(w - 1);
+    C[d] = static_cast<int32_t>(c);
+  }
+  return true;
+}
+
+radial_status build_mask(int32_t f, int32_t s, int32_t B, int32_t sink, int32_t dense, const MaskRule& rule,
                          radial_csr** out, cudaStream_t st) {
   const int64_t n64 = static_cast<int64_t>(f) * s;
   if (n64 > (1LL << 30)) return fail(RADIAL_EINVAL, "frames * tokens_per_frame = %lld exceeds 2^30", (long long)n64);
@@ -264,6 +312,22 @@ radial_status build_mask(int32_t f, int32_t s, int32_t B, int32_t sink, int32_t 
   if (!c) return fail(RADIAL_ENOMEM, "host allocation failed");
   c->f = f; c->s = s; c->n = n; c->B = B; c->sink = sink; c->dense = dense;
   cudaGetDevice(&c->device);
+  if (!rule.is_default()) {
+    std::vector<int32_t> H, C;
+    if (!mask_rule_table(rule, f, s, H, C)) {
+      delete c;
+      return fail(RADIAL_EUNSUPPORTED, "band table of width scale %d/%d overflows 128-bit arithmetic", rule.num,
+                  rule.den);
+    }
+    if (cudaMalloc(&c->hd, sizeof(int32_t) * f) != cudaSuccess || cudaMalloc(&c->cd, sizeof(int32_t) * f) != cudaSuccess) {
+      cudaFree(c->hd);
+      cudaFree(c->cd);
+      delete c;
+      return fail(RADIAL_ENOMEM, "cannot allocate the distance table");
+    }
+    cudaMemcpy(c->hd, H.data(), sizeof(int32_t) * f, cudaMemcpyHostToDevice);
+    cudaMemcpy(c->cd, C.data(), sizeof(int32_t) * f, cudaMemcpyHostToDevice);
+  }
   uint8_t* states = nullptr;
   uint8_t* states128 = nullptr;
   radial_status rs = RADIAL_OK;
@@ -275,13 +339,15 @@ radial_status build_mask(int32_t f, int32_t s, int32_t B, int32_t sink, int32_t 
       c->pairs.release();
       if (c->plan_owned) c->plan.release();
       c->user.release();
+      cudaFree(c->hd);
+      cudaFree(c->cd);
       delete c;
     }
     return r;
   };
   if (cudaMalloc(&states, static_cast<size_t>(nb) * nb) != cudaSuccess)
     return cleanup(fail(RADIAL_ENOMEM, "cannot allocate %d x %d tile states", nb, nb));
-  MaskGeom g{f, s, n, B, nb, sink};
+  MaskGeom g{f, s, n, B, nb, sink, c->hd, c->cd};
   dim3 grid((nb + 127) / 128, nb);
   classify_tiles_kernel<<<grid, 128, 0, st>>>(g, states);
   g_launches.fetch_add(1);
@@ -321,7 +387,9 @@ void radial_params_default(radial_params* p) {
   std::memset(p, 0, sizeof(*p));
   p->sink = 1;
   p->central_band = 1;
-  p->width_scale = 2;
+  p->width_scale_num = 2;
+  p->width_scale_den = 1;
+  p->decay = 0;
 }
 
 radial_status radial_mask_build(int32_t frames, int32_t tokens_per_frame, int32_t block,
@@ -331,14 +399,23 @@ radial_status radial_mask_build(int32_t frames, int32_t tokens_per_frame, int32_
   radial_params def;
   radial_params_default(&def);
   const radial_params* pr = params ? params : &def;
-  for (int i = 0; i < 5; ++i)
+  for (int i = 0; i < 3; ++i)
     if (pr->reserved[i] != 0) return fail(RADIAL_EINVAL, "params.reserved[%d] must be 0", i);
   if (pr->sink != 0 && pr->sink != 1) return fail(RADIAL_EINVAL, "params.sink must be 0 or 1");
-  if (pr->central_band != 1) return fail(RADIAL_EUNSUPPORTED, "only central_band = 1 is implemented");
-  if (pr->width_scale != 2) return fail(RADIAL_EUNSUPPORTED, "only width_scale = 2 is implemented");
+  if (pr->central_band < 0 || pr->central_band > (1 << 20))
+    return fail(RADIAL_EINVAL, "params.central_band must be in [0, 2^20]");
+  if (pr->width_scale_num < 1 || pr->width_scale_num > 64 || pr->width_scale_den < 1 || pr->width_scale_den > 64 ||
+      pr->width_scale_num <= pr->width_scale_den)
+    return fail(RADIAL_EINVAL, "width scale num/den must be in [1, 64] with num > den");
+  if (pr->decay != 0 && pr->decay != 1) return fail(RADIAL_EINVAL, "params.decay must be 0 (radial) or 1 (harmonic)");
+  MaskRule rule;
+  rule.central_band = pr->central_band;
+  rule.num = pr->width_scale_num;
+  rule.den = pr->width_scale_den;
+  rule.decay = pr->decay;
   if (frames < 1 || tokens_per_frame < 1) return fail(RADIAL_EINVAL, "frames and tokens_per_frame must be >= 1");
   if (block != 64 && block != 128) return fail(RADIAL_EUNSUPPORTED, "block must be 64 or 128");
-  return build_mask(frames, tokens_per_frame, block, pr->sink, 0, out, as_stream(stream));
+  return build_mask(frames, tokens_per_frame, block, pr->sink, 0, rule, out, as_stream(stream));
 }
 
 radial_status radial_mask_build_dense(int32_t n_tokens, int32_t block, radial_csr** out, void* stream) {
@@ -347,7 +424,7 @@ radial_status radial_mask_build_dense(int32_t n_tokens, int32_t block, radial_cs
   if (n_tokens < 1) return fail(RADIAL_EINVAL, "n_tokens must be >= 1");
   if (block != 64 && block != 128) return fail(RADIAL_EUNSUPPORTED, "block must be 64 or 128");
   // One frame of n tokens: distance 0 everywhere, so every pair is allowed.
-  return build_mask(1, n_tokens, block, 0, 1, out, as_stream(stream));
+  return build_mask(1, n_tokens, block, 0, 1, MaskRule(), out, as_stream(stream));
 }
 
 radial_status radial_csr_info(const radial_csr* c, radial_csr_info_t* info) {
@@ -385,6 +462,8 @@ radial_status radial_csr_copy_to_host(const radial_csr* c, int32_t* row_ptr, int
 void radial_csr_free(radial_csr* c) {
   if (!c) return;
   cudaDeviceSynchronize();
+  cudaFree(c->hd);
+  cudaFree(c->cd);
   c->pairs.release();
   if (c->plan_owned) c->plan.release();
   c->user.release();
@@ -465,6 +544,8 @@ radial_status launch_fwd_pair(const radial_csr* c, const radial_desc* d, const v
   p.pair_col = c->pairs.col;
   p.pair_flag = c->pairs.flag;
   p.pair_order = schedule_lpt() ? c->pairs.order : nullptr;
+  p.hd = c->hd;
+  p.cd = c->cd;
   p.np = c->pairs.np;
   p.nt = c->plan.nb;
   p.f = c->f;
@@ -500,6 +581,8 @@ radial_status launch_fwd(const radial_csr* c, const radial_desc* d, const void* 
   p.col_idx = c->plan.col_idx;
   p.kind = c->plan.kind;
   p.order = schedule_lpt() ? c->plan.row_order : nullptr;
+  p.hd = c->hd;
+  p.cd = c->cd;
   p.nt = c->plan.nb;
   p.f = c->f;
   p.s = c->s;
@@ -554,6 +637,8 @@ radial_status launch_bwd(const radial_csr* c, const radial_desc* d, const void* 
   p.row_idx = c->plan.row_idx;
   p.kind_t = c->plan.kind_t;
   p.col_order = schedule_lpt() ? c->plan.col_order : nullptr;
+  p.hd = c->hd;
+  p.cd = c->cd;
   p.nt = c->plan.nb;
   p.f = c->f;
   p.s = c->s;

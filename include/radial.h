@@ -51,19 +51,30 @@ typedef enum radial_status {
 } radial_status;
 
 /* Mask parameters.  sink: 1 = every query also attends to all tokens of frame
- * 0 (App. A.1 Eq.8; default 1).  central_band: frame distances <= this are
- * dense (the authors' "width of central band" ablation; only the default 1 is
- * implemented).  width_scale: width ratio between consecutive temporal bands
- * (their "width scale" ablation; only the default 2 is implemented).
- * reserved: must be zero. */
+ * 0 (App. A.1 Eq.8; default 1).  The remaining fields select the ablation
+ * variants of the authors' responses (paperhub.cn: "width of central band",
+ * "width scale between consecutive bands") and of the review's App. C.3
+ * (harmonic-series decay); their formulas are not printed, the readings are:
+ *  central_band (>= 0, default 1): frame distances <= it are dense.
+ *  width_scale_num / width_scale_den (sigma = num/den, 1 < sigma, both in
+ *    [1, 64], default 2/1): radial decay puts distance dist > cb in band r >= 1
+ *    with (cb+1) sigma^(r-1) <= dist < (cb+1) sigma^r and keeps
+ *    |k - l| <= floor(s / sigma^r) - 1.
+ *  decay (0 radial = the method, default; 1 harmonic): harmonic keeps
+ *    |k - l| <= floor(s / (dist - cb + 1)) - 1.
+ *  In both decays a width of 0 keeps only k == l, in every c-th frame pair,
+ *  c = ceil(sigma^r / s) (radial) or ceil((dist - cb + 1) / s) (harmonic).
+ * The defaults reproduce the method's mask exactly.  reserved: must be zero. */
 typedef struct radial_params {
   int32_t sink;
   int32_t central_band;
-  int32_t width_scale;
-  int32_t reserved[5];
+  int32_t width_scale_num;
+  int32_t width_scale_den;
+  int32_t decay;
+  int32_t reserved[3];
 } radial_params;
 
-/* Fill *p with the defaults {sink = 1, central_band = 1, width_scale = 2}. */
+/* Fill *p with the defaults {sink 1, central_band 1, width scale 2/1, decay radial}. */
 void radial_params_default(radial_params* p);
 
 /* Opaque block-sparse mask: the block CSR and CSC of active tiles plus the
@@ -94,9 +105,10 @@ typedef struct radial_csr_info_t {
  * Runs on the device on `stream` and SYNCHRONISES it (the tile count sizes the
  * allocation).  Constraints: f >= 1, s >= 1, f*s <= 2^30, B in {64, 128},
  * ceil(n/B) <= 32768.  On success *out owns device memory until
- * radial_csr_free.  Errors: RADIAL_EINVAL (bad sizes, null out/params,
- * non-zero reserved), RADIAL_EUNSUPPORTED (non-default central_band or
- * width_scale, other B), RADIAL_ENOMEM, RADIAL_ECUDA. */
+ * radial_csr_free.  params NULL selects the defaults.  Errors: RADIAL_EINVAL
+ * (bad sizes, null out, out-of-range or non-zero reserved parameters),
+ * RADIAL_EUNSUPPORTED (other B; a width scale whose band table would
+ * overflow 128-bit arithmetic), RADIAL_ENOMEM, RADIAL_ECUDA. */
 radial_status radial_mask_build(int32_t frames, int32_t tokens_per_frame, int32_t block,
                                 const radial_params* params, radial_csr** out, void* stream);
 

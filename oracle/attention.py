@@ -76,13 +76,13 @@ def backward(q, k, v, o, do, lse, allowed, scale):
 # Radial-mask wrappers over [B, H, N, D] arrays
 # ---------------------------------------------------------------------------
 
-def radial_forward(q, k, v, f, s, sink=True, scale=None):
+def radial_forward(q, k, v, f, s, sink=True, scale=None, spec=None):
     """Eq.2 under the radial mask for every (batch, head) of [B, H, N, D] inputs."""
     q, k, v = _as64(q), _as64(k), _as64(v)
     Bn, H, N, D = q.shape
     assert N == f * s
     scale = 1.0 / np.sqrt(D) if scale is None else scale
-    M = _mask.token_mask(f, s, sink)
+    M = _mask.token_mask(f, s, sink, spec)
     O = np.empty_like(q)
     L = np.empty((Bn, H, N))
     for b in range(Bn):
@@ -91,12 +91,12 @@ def radial_forward(q, k, v, f, s, sink=True, scale=None):
     return O, L
 
 
-def radial_backward(q, k, v, o, do, lse, f, s, sink=True, scale=None):
+def radial_backward(q, k, v, o, do, lse, f, s, sink=True, scale=None, spec=None):
     """Gradients under the radial mask for every (batch, head)."""
     q = _as64(q)
     Bn, H, N, D = q.shape
     scale = 1.0 / np.sqrt(D) if scale is None else scale
-    M = _mask.token_mask(f, s, sink)
+    M = _mask.token_mask(f, s, sink, spec)
     out = [np.empty_like(q) for _ in range(3)]
     for b in range(Bn):
         for h in range(H):

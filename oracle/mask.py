@@ -48,6 +48,8 @@ scales to the benchmark shapes; the tests pin the second to the first.
 
 from __future__ import annotations
 
+from dataclasses import dataclass
+
 import numpy as np
 
 TILE_FULL = 1
@@ -89,22 +91,88 @@ def distance_table(f, s):
 
 
 # ---------------------------------------------------------------------------
+# Ablation variants ([rebuttal]: width of the central band, width scale
+# between consecutive bands; [review] App. C.3: harmonic-series decay)
+# ---------------------------------------------------------------------------
+
+@dataclass(frozen=True)
+class MaskSpec:
+    """Mask family.  central_band: frame distances <= it are dense ([rebuttal]
+    "a central band width of d means attention between frames i and j where
+    |i - j| <= d", default 1).  Width scale sigma = scale_num / scale_den > 1
+    between consecutive temporal bands ([rebuttal], default 2).  decay:
+    "radial" (exponential bands, the method) or "harmonic" ([review] App. C.3:
+    width inversely proportional to the distance from the diagonal).
+
+    Readings (the pages print no formula for the variants):
+      radial:   dist <= cb -> dense; else band r >= 1 with
+                (cb+1) sigma^(r-1) <= dist < (cb+1) sigma^r, width
+                w = floor(s / sigma^r).  cb = 1, sigma = 2 gives exactly
+                r = floor(log2 dist), w = floor(s / 2^r) (the default rule).
+      harmonic: dist <= cb -> dense; else e = dist - cb + 1, w = floor(s / e).
+    In both, h = w - 1, and when w = 0 the diagonal k == l is kept in every
+    c-th frame pair, c = ceil(s_eff / s) with s_eff = sigma^r (radial) or e
+    (harmonic): the same amortised-density reading as the default."""
+
+    central_band: int = 1
+    scale_num: int = 2
+    scale_den: int = 1
+    decay: str = "radial"
+
+
+DEFAULT_SPEC = MaskSpec()
+
+
+def width_and_period(dist, s, spec=DEFAULT_SPEC):
+    """(w, c) of one frame distance, in exact integer / rational arithmetic."""
+    dist, s = int(dist), int(s)
+    cb = spec.central_band
+    if dist <= cb:
+        return s, 1
+    if spec.decay == "harmonic":
+        e = dist - cb + 1
+        w = s // e
+        return w, (1 if w >= 1 else -(-e // s))
+    p, q = spec.scale_num, spec.scale_den
+    # smallest r >= 1 with dist < (cb+1) (p/q)^r, i.e. dist * q^r < (cb+1) * p^r
+    r = 1
+    while not (dist * q ** r < (cb + 1) * p ** r):
+        r += 1
+    w = (s * q ** r) // (p ** r)                      # floor(s / sigma^r)
+    c = 1 if w >= 1 else -(-(p ** r) // (s * q ** r))  # ceil(sigma^r / s)
+    return w, c
+
+
+def spec_distance_table(f, s, spec=DEFAULT_SPEC):
+    """(h, c) for every frame distance in [0, f) under a mask spec."""
+    wc = [width_and_period(d, s, spec) for d in range(max(f, 1))]
+    h = np.array([w - 1 for w, _ in wc], dtype=np.int64)
+    c = np.array([c for _, c in wc], dtype=np.int64)
+    return h, c
+
+
+# ---------------------------------------------------------------------------
 # Token-level mask (Eq.4 + Eq.8, flattened)
 # ---------------------------------------------------------------------------
 
-def allowed(i, k, j, l, s, sink=True):
+def allowed(i, k, j, l, s, sink=True, spec=None):
     """Allowed(query frame i pos k, key frame j pos l); broadcasts over arrays.
 
     (sink and j == 0)  or  (h(d) >= 0 and |k-l| <= h(d))
                        or  (h(d) < 0 and d mod c(d) == 0 and k == l),  d = |i-j|.
+    spec None: the method's own rule (closed form); a MaskSpec: an ablation.
     """
     i = np.asarray(i, dtype=np.int64)
     j = np.asarray(j, dtype=np.int64)
     k = np.asarray(k, dtype=np.int64)
     l = np.asarray(l, dtype=np.int64)
     d = np.abs(i - j)
-    h = half_width(d, s)
-    c = sample_period(d, s)
+    if spec is None:
+        h = half_width(d, s)
+        c = sample_period(d, s)
+    else:
+        H, Cp = spec_distance_table(int(d.max()) + 1 if d.size else 1, s, spec)
+        h, c = H[d], Cp[d]
     band = (h >= 0) & (np.abs(k - l) <= h)
     sampled = (h < 0) & (d % c == 0) & (k == l)
     out = band | sampled
@@ -113,25 +181,25 @@ def allowed(i, k, j, l, s, sink=True):
     return out
 
 
-def allowed_tokens(a, b, s, sink=True):
+def allowed_tokens(a, b, s, sink=True, spec=None):
     """allowed() on flat token indices a (query) and b (key)."""
     a = np.asarray(a, dtype=np.int64)
     b = np.asarray(b, dtype=np.int64)
-    return allowed(a // s, a % s, b // s, b % s, s, sink)
+    return allowed(a // s, a % s, b // s, b % s, s, sink, spec)
 
 
-def token_mask(f, s, sink=True):
+def token_mask(f, s, sink=True, spec=None):
     """Dense n x n boolean mask (True = allowed).  Tiny shapes only."""
     n = f * s
     a = np.arange(n, dtype=np.int64)
-    return allowed_tokens(a[:, None], a[None, :], s, sink)
+    return allowed_tokens(a[:, None], a[None, :], s, sink, spec)
 
 
-def _mask_from_table(qi, qk, kj, kl, f, s, sink):
+def _mask_from_table(qi, qk, kj, kl, f, s, sink, spec=None):
     """allowed() over a (queries x keys) grid using the per-distance table
     (h(d), c(d)) of distance_table() instead of recomputing it per pair.
     Same predicate, int32 arithmetic."""
-    H, Cp = distance_table(f, s)
+    H, Cp = distance_table(f, s) if spec is None else spec_distance_table(f, s, spec)
     H = H.astype(np.int32)
     Cp = Cp.astype(np.int32)
     d = np.abs(qi[:, None] - kj[None, :])
@@ -145,32 +213,32 @@ def _mask_from_table(qi, qk, kj, kl, f, s, sink):
     return out
 
 
-def row_mask(rows, f, s, sink=True):
+def row_mask(rows, f, s, sink=True, spec=None):
     """Boolean mask of the given query rows against all n keys."""
     n = f * s
     rows = np.asarray(rows, dtype=np.int32)
     b = np.arange(n, dtype=np.int32)
-    return _mask_from_table(rows // s, rows % s, b // s, b % s, f, s, sink)
+    return _mask_from_table(rows // s, rows % s, b // s, b % s, f, s, sink, spec)
 
 
-def col_mask(cols, f, s, sink=True):
+def col_mask(cols, f, s, sink=True, spec=None):
     """Boolean mask of all n queries against the given key columns (n x len)."""
     n = f * s
     cols = np.asarray(cols, dtype=np.int32)
     a = np.arange(n, dtype=np.int32)
-    return _mask_from_table(a // s, a % s, cols // s, cols % s, f, s, sink)
+    return _mask_from_table(a // s, a % s, cols // s, cols % s, f, s, sink, spec)
 
 
 # ---------------------------------------------------------------------------
 # Block tiles: brute force
 # ---------------------------------------------------------------------------
 
-def tile_states_bruteforce(f, s, B, sink=True):
+def tile_states_bruteforce(f, s, B, sink=True, spec=None):
     """uint8 [nb, nb]: 0 inactive, TILE_FULL, TILE_PARTIAL -- from the token mask."""
     n = f * s
     nb = -(-n // B)
     m = np.zeros((nb * B, nb * B), dtype=bool)
-    m[:n, :n] = token_mask(f, s, sink)
+    m[:n, :n] = token_mask(f, s, sink, spec)
     t = m.reshape(nb, B, nb, B)
     active = t.any(axis=(1, 3))
     every = t.all(axis=(1, 3))
@@ -209,7 +277,7 @@ def _segments(nb, B, n, s):
     return frame, lo, hi, valid
 
 
-def tile_states_intervals(f, s, B, sink=True, chunk=64):
+def tile_states_intervals(f, s, B, sink=True, chunk=64, spec=None):
     """uint8 [nb, nb] tile states from the interval test.
 
     For a query segment (frame i, positions [k0, k1]) and a key segment
@@ -225,6 +293,8 @@ def tile_states_intervals(f, s, B, sink=True, chunk=64):
     nb = -(-n // B)
     fr, lo, hi, va = _segments(nb, B, n, s)
     inside = (np.arange(nb) + 1) * B <= n
+    if spec is not None:
+        Ht, Ct = spec_distance_table(f, s, spec)
     out = np.zeros((nb, nb), dtype=np.uint8)
     # key-side arrays broadcast as [1, 1, nb, S]
     jf, l0, l1, jv = (x[None, None] for x in (fr, lo, hi, va))
@@ -232,8 +302,12 @@ def tile_states_intervals(f, s, B, sink=True, chunk=64):
         q1 = min(nb, q0 + chunk)
         i_, k0, k1, iv = (x[q0:q1, :, None, None] for x in (fr, lo, hi, va))
         d = np.abs(i_ - jf)
-        h = half_width(d, s)
-        c = sample_period(d, s)
+        if spec is None:
+            h = half_width(d, s)
+            c = sample_period(d, s)
+        else:
+            dd = np.minimum(d, f - 1)      # distances >= f only occur on invalid segments
+            h, c = Ht[dd], Ct[dd]
         gap = np.maximum(0, np.maximum(l0 - k1, k0 - l1))
         span = np.maximum(k1 - l0, l1 - k0)
         band_any = (h >= 0) & (gap <= h)
@@ -285,12 +359,12 @@ def row_order(row_ptr):
     return np.lexsort((idx, -counts)).astype(np.int32)
 
 
-def block_csr(f, s, B, sink=True, method="intervals"):
+def block_csr(f, s, B, sink=True, method="intervals", spec=None):
     """Everything the block-sparse executor needs, as a dict of numpy arrays."""
     if method == "bruteforce":
-        st = tile_states_bruteforce(f, s, B, sink)
+        st = tile_states_bruteforce(f, s, B, sink, spec)
     else:
-        st = tile_states_intervals(f, s, B, sink)
+        st = tile_states_intervals(f, s, B, sink, spec=spec)
     row_ptr, col_idx, kind = csr_from_states(st)
     col_ptr, row_idx, kind_t = csc_from_states(st)
     return dict(
@@ -305,7 +379,7 @@ def block_csr(f, s, B, sink=True, method="intervals"):
 # Pair counting (complexity invariants, [review] §4.2 Eq.5/Eq.6)
 # ---------------------------------------------------------------------------
 
-def allowed_pair_count(f, s, sink=True):
+def allowed_pair_count(f, s, sink=True, spec=None):
     """Number of allowed (query, key) token pairs, summed per frame pair.
 
     Counts positions directly per frame pair: for each (i, j) build the s x s
@@ -316,5 +390,5 @@ def allowed_pair_count(f, s, sink=True):
     total = 0
     for i in range(f):
         for j in range(f):
-            total += int(allowed(i, k, j, l, s, sink).sum())
+            total += int(allowed(i, k, j, l, s, sink, spec).sum())
     return total

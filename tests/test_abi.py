@@ -48,8 +48,8 @@ def test_symbols_are_c_linkage():
 
 def test_params_default(lib):
     p = rb.radial_params_default()
-    assert (p.sink, p.central_band, p.width_scale) == (1, 1, 2)
-    assert list(p.reserved) == [0] * 5
+    assert (p.sink, p.central_band, p.width_scale_num, p.width_scale_den, p.decay) == (1, 1, 2, 1, 0)
+    assert list(p.reserved) == [0] * 3
 
 
 def test_status_strings(lib):
@@ -61,8 +61,10 @@ def test_status_strings(lib):
     (dict(frames=0, tokens_per_frame=4, block=64), 1),
     (dict(frames=4, tokens_per_frame=0, block=64), 1),
     (dict(frames=4, tokens_per_frame=4, block=96), 2),
-    (dict(frames=4, tokens_per_frame=4, block=128, central_band=2), 2),
-    (dict(frames=4, tokens_per_frame=4, block=128, width_scale=3), 2),
+    (dict(frames=4, tokens_per_frame=4, block=128, central_band=-1), 1),
+    (dict(frames=4, tokens_per_frame=4, block=128, width_scale=(2, 2)), 1),
+    (dict(frames=4, tokens_per_frame=4, block=128, width_scale=(65, 1)), 1),
+    (dict(frames=4, tokens_per_frame=4, block=128, decay=2), 1),
     (dict(frames=4, tokens_per_frame=4, block=128, sink=7), 1),
     (dict(frames=4, tokens_per_frame=4, block=128, reserved=[0, 0, 1]), 1),
     (dict(frames=1 << 16, tokens_per_frame=1 << 16, block=128), 1),
