@@ -333,31 +333,38 @@ __global__ void __launch_bounds__(384, 1)
           else
             mw[0] = mw[1] = mw[2] = mw[3] = 0u;
         }
+        const uint32_t modes = partial ? chunk_modes(mw) : 0u;
         mbar_wait(&bars->s_full, g & 1, abort_flag);
         __syncwarp();
         tc_fence_after();
 #pragma unroll
         for (int c = 0; c < 2; ++c) {
           const int gc = 2 * wg + c;  // 32-column chunk of the tile
-          uint32_t rs[32], rp[32];
-          tmem_ld32(tmem + lane_addr + TM_S + gc * 32, rs);
-          tmem_ld32(tmem + lane_addr + TM_DP + gc * 32, rp);
-          tmem_wait_ld();
-          const uint32_t bits = mw[gc];
+          const uint32_t mode = (modes >> (2 * gc)) & 3u;
           uint32_t pw[16], dw[16];
+          if (mode == 2u) {  // every lane of the warp masks this chunk: P^T = dS^T = 0
 #pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            float pv[2], dv[2];
+            for (int e = 0; e < 16; ++e) pw[e] = dw[e] = 0u;
+          } else {
+            uint32_t rs[32], rp[32];
+            tmem_ld32(tmem + lane_addr + TM_S + gc * 32, rs);
+            tmem_ld32(tmem + lane_addr + TM_DP + gc * 32, rp);
+            tmem_wait_ld();
+            const uint32_t bits = mode == 0u ? 0xffffffffu : mw[gc];
 #pragma unroll
-            for (int z = 0; z < 2; ++z) {
-              const int ql = c * 32 + 2 * e + z;  // query index inside this warpgroup's 64
-              const bool ok = (bits >> (2 * e + z)) & 1u;
-              const float x = fmaf(__uint_as_float(rs[2 * e + z]), p.scale_log2, -vbuf[ql]);
-              pv[z] = ok ? ex2_approx(x) : 0.f;
-              dv[z] = pv[z] * (__uint_as_float(rp[2 * e + z]) - vbuf[64 + ql]);
+            for (int e = 0; e < 16; ++e) {
+              float pv[2], dv[2];
+#pragma unroll
+              for (int z = 0; z < 2; ++z) {
+                const int ql = c * 32 + 2 * e + z;  // query index inside this warpgroup's 64
+                const float x = fmaf(__uint_as_float(rs[2 * e + z]), p.scale_log2, -vbuf[ql]);
+                pv[z] = ex2_approx(x);
+                if (mode != 0u) pv[z] = ((bits >> (2 * e + z)) & 1u) ? pv[z] : 0.f;
+                dv[z] = pv[z] * (__uint_as_float(rp[2 * e + z]) - vbuf[64 + ql]);
+              }
+              pw[e] = pack_bf16x2(pv[0], pv[1]);
+              dw[e] = pack_bf16x2(dv[0], dv[1]);
             }
-            pw[e] = pack_bf16x2(pv[0], pv[1]);
-            dw[e] = pack_bf16x2(dv[0], dv[1]);
           }
           // bf16 results go to this warpgroup's own columns, over data already read
           tmem_st16(tmem + lane_addr + TM_S + 64 * wg + c * 16, pw);
@@ -581,28 +588,35 @@ __global__ void __launch_bounds__(384, 1)
           mbar_wait(&bars->mma2_done[db], ((g >> 1) - 1) & 1, abort_flag);
           __syncwarp();
         }
+        const uint32_t modes = partial ? chunk_modes(mw) : 0u;
         mbar_wait(&bars->s_full, g & 1, abort_flag);
         __syncwarp();
         tc_fence_after();
 #pragma unroll
         for (int c = 0; c < 2; ++c) {
           const int gc = 2 * wg + c;
-          uint32_t rs[32], rp[32];
-          tmem_ld32(tmem + lane_addr + TM_S + gc * 32, rs);
-          tmem_ld32(tmem + lane_addr + TM_DP + gc * 32, rp);
-          tmem_wait_ld();
-          const uint32_t bits = mw[gc];
+          const uint32_t mode = (modes >> (2 * gc)) & 3u;
           uint32_t dw[16];
+          if (mode == 2u) {  // every lane of the warp masks this chunk: dS = 0
 #pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            float dv[2];
+            for (int e = 0; e < 16; ++e) dw[e] = 0u;
+          } else {
+            uint32_t rs[32], rp[32];
+            tmem_ld32(tmem + lane_addr + TM_S + gc * 32, rs);
+            tmem_ld32(tmem + lane_addr + TM_DP + gc * 32, rp);
+            tmem_wait_ld();
+            const uint32_t bits = mw[gc];
 #pragma unroll
-            for (int z = 0; z < 2; ++z) {
-              const bool ok = (bits >> (2 * e + z)) & 1u;
-              const float pv = ok ? ex2_approx(fmaf(__uint_as_float(rs[2 * e + z]), p.scale_log2, -lse2)) : 0.f;
-              dv[z] = pv * (__uint_as_float(rp[2 * e + z]) - drow);
+            for (int e = 0; e < 16; ++e) {
+              float dv[2];
+#pragma unroll
+              for (int z = 0; z < 2; ++z) {
+                float pv = ex2_approx(fmaf(__uint_as_float(rs[2 * e + z]), p.scale_log2, -lse2));
+                if (mode != 0u) pv = ((bits >> (2 * e + z)) & 1u) ? pv : 0.f;
+                dv[z] = pv * (__uint_as_float(rp[2 * e + z]) - drow);
+              }
+              dw[e] = pack_bf16x2(dv[0], dv[1]);
             }
-            dw[e] = pack_bf16x2(dv[0], dv[1]);
           }
           tmem_st16(tmem + lane_addr + TM_DS + db * 64 + gc * 16, dw);
         }

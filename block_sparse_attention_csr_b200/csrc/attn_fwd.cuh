@@ -98,12 +98,21 @@ __device__ __forceinline__ void set_bits(uint32_t (&mw)[4], int lo, int hi) {
   }
 }
 
+// floor(x / s) for 0 <= x < 2^30 without an integer division: a float
+// estimate from the reciprocal, then an exact correction of at most one step.
+__device__ __forceinline__ int div_by(int x, int s) {
+  int q = __float2int_rz(static_cast<float>(x) * __frcp_rn(static_cast<float>(s)));
+  q += (q + 1) * s <= x;
+  q -= q * s > x;
+  return q;
+}
+
 // Allowed key columns (relative to b0, 128 wide) of query token a = i*s + k.
 __device__ __forceinline__ void row_mask_bits(const FwdParams& p, int i, int k, int b0,
                                               uint32_t (&mw)[4]) {
   mw[0] = mw[1] = mw[2] = mw[3] = 0u;
   const int bend = min(b0 + 128, p.n);  // exclusive
-  for (int j = b0 / p.s; j * p.s < bend; ++j) {
+  for (int j = div_by(b0, p.s); j * p.s < bend; ++j) {
     const int seg_lo = max(b0, j * p.s) - b0;
     const int seg_hi = min(bend, (j + 1) * p.s) - 1 - b0;
     int lo, hi;
@@ -128,10 +137,41 @@ __device__ __forceinline__ void row_mask_bits(const FwdParams& p, int i, int k, 
   }
 }
 
-// kFastSoftmax: tree reductions, packed fp32x2 FMA / add, and every
-// kPolyEvery-th pair of exponentials on the FMA pipe (exp2_poly_x2) to take
-// load off the MUFU pipe; otherwise the plain one-MUFU-per-element loop.
-constexpr int kPolyEvery = 4;
+// kFastSoftmax: tree reductions and packed fp32x2 FMA / add; otherwise the
+// plain serial loop.  kPolyEvery > 0 computes every kPolyEvery-th pair of
+// exponentials on the FMA pipe (exp2_poly_x2) instead of the MUFU.  Measured
+// on B200 the softmax is issue-bound, not MUFU-bound (moving a quarter of the
+// exponentials to the polynomial made the forward 4-5 % slower, half of them
+// 13 %), so it is off.
+constexpr int kPolyEvery = 0;
+__host__ __device__ constexpr bool use_poly_exp(int e) {
+  return kPolyEvery > 0 && (e % (kPolyEvery > 0 ? kPolyEvery : 1)) == kPolyEvery - 1;
+}
+
+// Warp-uniform handling of one 32-column chunk of a PARTIAL tile: 0 = every
+// lane of the warp allows all 32 columns (use S as is), 2 = every lane masks
+// all of them (no TMEM read, no select, no exponential: P = 0), 1 = mixed
+// (per-element select).  Two bits per chunk.
+__device__ __forceinline__ uint32_t chunk_modes(const uint32_t (&mw)[4]) {
+  uint32_t modes = 0;
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {
+    const bool all_ok = __all_sync(0xffffffffu, mw[c] == 0xffffffffu);
+    const bool none = __all_sync(0xffffffffu, mw[c] == 0u);
+    modes |= (all_ok ? 0u : (none ? 2u : 1u)) << (2 * c);
+  }
+  return modes;
+}
+
+// Applies a chunk's mask in place to the raw fp32 bits of S (a fully masked
+// chunk has word 0, so the select gives -inf there too).
+__device__ __forceinline__ void mask_chunk_inplace(uint32_t (&r)[32], uint32_t word, uint32_t mode) {
+  constexpr uint32_t kNegInf = 0xff800000u;
+  if (mode != 0u) {
+#pragma unroll
+    for (int e = 0; e < 32; ++e) r[e] = ((word >> e) & 1u) ? r[e] : kNegInf;
+  }
+}
 
 template <int D, bool kFastSoftmax>
 __global__ void __launch_bounds__(192, 1)
@@ -378,7 +418,7 @@ __global__ void __launch_bounds__(192, 1)
               const int i0 = c * 64 + 2 * e;
               const uint64_t x = f2_fma(f2_pack(sv[i0], sv[i0 + 1]), sl2, negm);
               uint64_t pe;
-              if ((e % kPolyEvery) == kPolyEvery - 1) {
+              if (use_poly_exp(e)) {
                 pe = exp2_poly_x2(x);
               } else {
                 float x0, x1;
