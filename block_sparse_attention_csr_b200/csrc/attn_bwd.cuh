@@ -237,7 +237,12 @@ __global__ void __launch_bounds__(384, 1)
     if (lane == 0) {
       constexpr uint32_t idesc_s = idesc_bf16_f32(128, 128, false, false);
       constexpr uint32_t idesc_g = idesc_bf16_f32(128, D, false, true);
-      const uint32_t k_base = smem_u32(sK), v_base = smem_u32(sV), q_base = smem_u32(sQ);
+      // descriptors built once; stages and K-steps are offsets (see the forward)
+      constexpr uint64_t kTile = C::TILE_BYTES >> 4;
+      const uint64_t dK = smem_desc(smem_u32(sK), 16, 1024, kSwizzle128B);
+      const uint64_t dV = smem_desc(smem_u32(sV), 16, 1024, kSwizzle128B);
+      const uint64_t dQk = smem_desc(smem_u32(sQ), 16, 1024, kSwizzle128B);       // Q, dO as K-major B
+      const uint64_t dQmn = smem_desc(smem_u32(sQ), 16384, 1024, kSwizzle128B);   // Q, dO as MN-major B
       uint32_t it = 0, item_i = 0;
       for (int item = blockIdx.x; item < p.items; item += gridDim.x, ++item_i) {
         const int bh = item / p.nt;
@@ -248,39 +253,33 @@ __global__ void __launch_bounds__(384, 1)
         for (uint32_t j = 0; j < n_tiles; ++j) {
           const uint32_t g = it + j, st = g % C::STAGES;
           mbar_wait(&bars->st_full[st], (g / C::STAGES) & 1, abort_flag);
-          // S^T / dP^T columns still hold P^T / dS^T of the previous tile until
-          // its dV / dK MMAs have completed.
-          if (g >= 1) mbar_wait(&bars->mma2_done[(g - 1) & 1], ((g - 1) >> 1) & 1, abort_flag);
           tc_fence_after();
-          const uint32_t qb = q_base + st * 2 * C::TILE_BYTES, ob = qb + C::TILE_BYTES;
+          // S^T / dP^T overwrite the columns where P^T / dS^T of tile g-1 are read
+          // by its dV / dK MMAs, issued just before in the same MMA stream.
+          const uint64_t qk = dQk + st * 2 * kTile, ok = qk + kTile;
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-            mma_ss(tmem + TM_S, smem_desc(k_base + off, 16, 1024, kSwizzle128B),
-                   smem_desc(qb + off, 16, 1024, kSwizzle128B), idesc_s, kk > 0 ? 1u : 0u);
+            const uint64_t off = static_cast<uint64_t>(((kk >> 2) * 16384 + (kk & 3) * 32) >> 4);
+            mma_ss(tmem + TM_S, dK + off, qk + off, idesc_s, kk > 0 ? 1u : 0u);
           }
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-            mma_ss(tmem + TM_DP, smem_desc(v_base + off, 16, 1024, kSwizzle128B),
-                   smem_desc(ob + off, 16, 1024, kSwizzle128B), idesc_s, kk > 0 ? 1u : 0u);
+            const uint64_t off = static_cast<uint64_t>(((kk >> 2) * 16384 + (kk & 3) * 32) >> 4);
+            mma_ss(tmem + TM_DP, dV + off, ok + off, idesc_s, kk > 0 ? 1u : 0u);
           }
           mma_commit(&bars->s_full);
           mbar_wait(&bars->ew_full[g & 1], (g >> 1) & 1, abort_flag);
           if (j == 0 && item_i > 0) mbar_wait(&bars->acc_empty, (item_i - 1) & 1, abort_flag);
           tc_fence_after();
+          const uint64_t qmn = dQmn + st * 2 * kTile, omn = qmn + kTile;
 #pragma unroll
-          for (int kk = 0; kk < 8; ++kk) {  // K = 128 query rows, 16 per MMA
-            mma_ts(tmem + TM_DV, tmem + TM_S + 64 * (kk >> 2) + 8 * (kk & 3),
-                   smem_desc(ob + kk * 2048, 16384, 1024, kSwizzle128B),
-                   idesc_g, (j > 0 || kk > 0) ? 1u : 0u);
-          }
+          for (int kk = 0; kk < 8; ++kk)  // K = 128 query rows, 16 per MMA
+            mma_ts(tmem + TM_DV, tmem + TM_S + 64 * (kk >> 2) + 8 * (kk & 3), omn + kk * (2048 >> 4), idesc_g,
+                   (j > 0 || kk > 0) ? 1u : 0u);
 #pragma unroll
-          for (int kk = 0; kk < 8; ++kk) {
-            mma_ts(tmem + TM_DK, tmem + TM_DP + 64 * (kk >> 2) + 8 * (kk & 3),
-                   smem_desc(qb + kk * 2048, 16384, 1024, kSwizzle128B),
-                   idesc_g, (j > 0 || kk > 0) ? 1u : 0u);
-          }
+          for (int kk = 0; kk < 8; ++kk)
+            mma_ts(tmem + TM_DK, tmem + TM_DP + 64 * (kk >> 2) + 8 * (kk & 3), qmn + kk * (2048 >> 4), idesc_g,
+                   (j > 0 || kk > 0) ? 1u : 0u);
           mma_commit(&bars->mma2_done[g & 1]);
           mma_commit(&bars->st_empty[st]);
           if (j + 1 == n_tiles) mma_commit(&bars->fix_empty);
@@ -497,18 +496,22 @@ __global__ void __launch_bounds__(384, 1)
     if (lane == 0) {
       constexpr uint32_t idesc_s = idesc_bf16_f32(128, 128, false, false);
       constexpr uint32_t idesc_g = idesc_bf16_f32(128, D, false, true);
-      const uint32_t q_base = smem_u32(sQ), o_base = smem_u32(sdO), k_base = smem_u32(sK);
+      constexpr uint64_t kTile = C::TILE_BYTES >> 4;
+      const uint64_t dQ = smem_desc(smem_u32(sQ), 16, 1024, kSwizzle128B);
+      const uint64_t dO = smem_desc(smem_u32(sdO), 16, 1024, kSwizzle128B);
+      const uint64_t dKk = smem_desc(smem_u32(sK), 16, 1024, kSwizzle128B);       // K, V as K-major B
+      const uint64_t dKmn = smem_desc(smem_u32(sK), 16384, 1024, kSwizzle128B);   // K as MN-major B
       uint32_t it = 0, item_i = 0;
       auto issue_dq = [&](uint32_t g, uint32_t j) {
         const uint32_t st = g % C::STAGES, db = g & 1;
         mbar_wait(&bars->ew_full[db], (g >> 1) & 1, abort_flag);
         if (j == 0 && item_i > 0) mbar_wait(&bars->acc_empty, (item_i - 1) & 1, abort_flag);
         tc_fence_after();
-        const uint32_t kb = k_base + st * 2 * C::TILE_BYTES;
+        const uint64_t kmn = dKmn + st * 2 * kTile;
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
-          mma_ts(tmem + TM_DQ, tmem + TM_DS + db * 64 + kk * 8,
-                 smem_desc(kb + kk * 2048, 16384, 1024, kSwizzle128B), idesc_g, (j > 0 || kk > 0) ? 1u : 0u);
+          mma_ts(tmem + TM_DQ, tmem + TM_DS + db * 64 + kk * 8, kmn + kk * (2048 >> 4), idesc_g,
+                 (j > 0 || kk > 0) ? 1u : 0u);
         mma_commit(&bars->mma2_done[db]);
         mma_commit(&bars->st_empty[st]);
       };
@@ -523,18 +526,16 @@ __global__ void __launch_bounds__(384, 1)
           mbar_wait(&bars->st_full[st], (g / C::STAGES) & 1, abort_flag);
           if (g >= 1) mbar_wait(&bars->s_free, (g - 1) & 1, abort_flag);
           tc_fence_after();
-          const uint32_t kb = k_base + st * 2 * C::TILE_BYTES, vb = kb + C::TILE_BYTES;
+          const uint64_t kk_ = dKk + st * 2 * kTile, vk = kk_ + kTile;
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-            mma_ss(tmem + TM_S, smem_desc(q_base + off, 16, 1024, kSwizzle128B),
-                   smem_desc(kb + off, 16, 1024, kSwizzle128B), idesc_s, kk > 0 ? 1u : 0u);
+            const uint64_t off = static_cast<uint64_t>(((kk >> 2) * 16384 + (kk & 3) * 32) >> 4);
+            mma_ss(tmem + TM_S, dQ + off, kk_ + off, idesc_s, kk > 0 ? 1u : 0u);
           }
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-            mma_ss(tmem + TM_DP, smem_desc(o_base + off, 16, 1024, kSwizzle128B),
-                   smem_desc(vb + off, 16, 1024, kSwizzle128B), idesc_s, kk > 0 ? 1u : 0u);
+            const uint64_t off = static_cast<uint64_t>(((kk >> 2) * 16384 + (kk & 3) * 32) >> 4);
+            mma_ss(tmem + TM_DP, dO + off, vk + off, idesc_s, kk > 0 ? 1u : 0u);
           }
           mma_commit(&bars->s_full);
           if (j + 1 == n_tiles) mma_commit(&bars->fix_empty);

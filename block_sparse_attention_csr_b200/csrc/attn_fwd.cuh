@@ -264,7 +264,11 @@ __global__ void __launch_bounds__(192, 1)
     if (lane == 0) {
       constexpr uint32_t idesc_s = idesc_bf16_f32(128, 128, false, false);
       constexpr uint32_t idesc_o = idesc_bf16_f32(128, D, false, true);
-      const uint32_t q_base = smem_u32(sQ), k_base = smem_u32(sK), v_base = smem_u32(sV);
+      // descriptors built once; stages and K-steps are start-address offsets
+      constexpr uint64_t kTile = C::TILE_BYTES >> 4;
+      const uint64_t dQ = smem_desc(smem_u32(sQ), 16, 1024, kSwizzle128B);
+      const uint64_t dK0 = smem_desc(smem_u32(sK), 16, 1024, kSwizzle128B);
+      const uint64_t dV0 = smem_desc(smem_u32(sV), 16384, 1024, kSwizzle128B);
       uint32_t it = 0, item_i = 0;
       auto issue_pv = [&](uint32_t g, uint32_t j) {
         const uint32_t st = g % C::STAGES, pb = g & 1;
@@ -272,13 +276,11 @@ __global__ void __launch_bounds__(192, 1)
         mbar_wait(&bars->v_full[st], (g / C::STAGES) & 1, abort_flag);
         if (j == 0 && item_i > 0) mbar_wait(&bars->o_empty, (item_i - 1) & 1, abort_flag);
         tc_fence_after();
-        const uint32_t vb = v_base + st * C::TILE_BYTES;
+        const uint64_t dv = dV0 + st * kTile;
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint64_t bdesc = smem_desc(vb + kk * 2048, 16384, 1024, kSwizzle128B);
-          mma_ts(tmem + C::TM_O, tmem + C::TM_P0 + pb * 64 + kk * 8, bdesc, idesc_o,
+        for (int kk = 0; kk < 8; ++kk)
+          mma_ts(tmem + C::TM_O, tmem + C::TM_P0 + pb * 64 + kk * 8, dv + kk * (2048 >> 4), idesc_o,
                  (j > 0 || kk > 0) ? 1u : 0u);
-        }
         mma_commit(&bars->pv_done[pb]);
         mma_commit(&bars->kv_empty[st]);
       };
@@ -294,13 +296,11 @@ __global__ void __launch_bounds__(192, 1)
           mbar_wait(&bars->k_full[st], (g / C::STAGES) & 1, abort_flag);
           if (g >= 2) mbar_wait(&bars->s_empty[sb], ((g >> 1) - 1) & 1, abort_flag);
           tc_fence_after();
-          const uint32_t kbase = k_base + st * C::TILE_BYTES;
+          const uint64_t dk = dK0 + st * kTile;
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-            const uint64_t adesc = smem_desc(q_base + off, 16, 1024, kSwizzle128B);
-            const uint64_t bdesc = smem_desc(kbase + off, 16, 1024, kSwizzle128B);
-            mma_ss(tmem + C::TM_S0 + sb * 128, adesc, bdesc, idesc_s, kk > 0 ? 1u : 0u);
+            const uint64_t off = static_cast<uint64_t>(((kk >> 2) * 16384 + (kk & 3) * 32) >> 4);
+            mma_ss(tmem + C::TM_S0 + sb * 128, dQ + off, dk + off, idesc_s, kk > 0 ? 1u : 0u);
           }
           mma_commit(&bars->s_full[sb]);
           if (j + 1 == n_tiles) mma_commit(&bars->q_empty);

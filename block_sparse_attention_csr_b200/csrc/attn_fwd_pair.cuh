@@ -183,10 +183,19 @@ __global__ void __launch_bounds__(384, 1)
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
+    // The issuing thread is the tensor pipe's only feeder: every instruction
+    // between two tcgen05.mma delays the pipe.  All shared-memory descriptors
+    // are therefore built once; a slot or K-step is a compile-time offset
+    // added to the start-address field (addresses stay below 256 KB, so the
+    // 14-bit field never carries).
     if (lane == 0) {
       constexpr uint32_t idesc_s = idesc_bf16_f32(128, 128, false, false);
       constexpr uint32_t idesc_o = idesc_bf16_f32(128, D, false, true);
-      const uint32_t q_base = smem_u32(sQ), k_base = smem_u32(sK), v_base = smem_u32(sV);
+      constexpr uint64_t kSlot = C::TILE_BYTES >> 4;  // one tile, in descriptor units
+      const uint64_t dq0 = smem_desc(smem_u32(sQ), 16, 1024, kSwizzle128B);
+      const uint64_t dk0 = smem_desc(smem_u32(sK), 16, 1024, kSwizzle128B);
+      const uint64_t dv0 = smem_desc(smem_u32(sV), 16384, 1024, kSwizzle128B);
+      const uint32_t tS = tmem + C::TM_S, tO = tmem + C::TM_O;
       uint32_t kc = 0, vc = 0, item_i = 0;
       uint32_t g[2] = {0u, 0u};       // S tiles issued per query tile (all items)
       uint32_t icnt[2] = {0u, 0u};    // items completed per query tile
@@ -207,12 +216,11 @@ __global__ void __launch_bounds__(384, 1)
           mbar_wait(&bars->v_full[vs], (vslot_count >> 1) & 1, abort_flag);
           if (first_pv[i] && icnt[i] > 0) mbar_wait(&bars->o_empty[i], (icnt[i] - 1) & 1, abort_flag);
           tc_fence_after();
-          const uint32_t vb = v_base + vs * C::TILE_BYTES;
+          const uint64_t dv = dv0 + vs * kSlot;
+          const uint32_t tPi = tS + i * 128, tOi = tO + i * 128;
+          mma_ts(tOi, tPi, dv, idesc_o, first_pv[i] ? 0u : 1u);
 #pragma unroll
-          for (int kk = 0; kk < 8; ++kk)
-            mma_ts(tmem + C::TM_O + i * 128, tmem + C::TM_S + i * 128 + kk * 8,
-                   smem_desc(vb + kk * 2048, 16384, 1024, kSwizzle128B), idesc_o,
-                   (!first_pv[i] || kk > 0) ? 1u : 0u);
+          for (int kk = 1; kk < 8; ++kk) mma_ts(tOi, tPi + kk * 8, dv + kk * (2048 >> 4), idesc_o, 1u);
           first_pv[i] = false;
           pending[i] = false;
         };
@@ -223,17 +231,18 @@ __global__ void __launch_bounds__(384, 1)
           const uint32_t ks = kc % C::K_SLOTS;
           mbar_wait(&bars->k_full[ks], (kc / C::K_SLOTS) & 1, abort_flag);
           tc_fence_after();
-          const uint32_t kb = k_base + ks * C::TILE_BYTES;
+          const uint64_t dk = dk0 + ks * kSlot;
 #pragma unroll
           for (int i = 0; i < 2; ++i) {
             if (pending[i]) issue_pv(i, vc - 1);  // V of the previous column
             if (fl & (i == 0 ? kPairIn0 : kPairIn1)) {
-              const uint32_t qb = q_base + i * C::TILE_BYTES;
+              const uint64_t dq = dq0 + i * kSlot;
+              const uint32_t tSi = tS + i * 128;
 #pragma unroll
               for (int kk = 0; kk < D / 16; ++kk) {
-                const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-                mma_ss(tmem + C::TM_S + i * 128, smem_desc(qb + off, 16, 1024, kSwizzle128B),
-                       smem_desc(kb + off, 16, 1024, kSwizzle128B), idesc_s, kk > 0 ? 1u : 0u);
+                constexpr uint64_t z = 0;
+                const uint64_t off = z + (((kk >> 2) * 16384 + (kk & 3) * 32) >> 4);
+                mma_ss(tSi, dq + off, dk + off, idesc_s, kk > 0 ? 1u : 0u);
               }
               mma_commit(&bars->s_full[i]);
               pending[i] = true;
