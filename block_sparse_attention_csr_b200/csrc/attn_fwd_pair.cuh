@@ -21,11 +21,11 @@
 //               tile's two MMAs (1024 tensor cycles) to turn S into P.
 //   warps 4-7   softmax warpgroup of tile 0, warps 8-11 of tile 1: one thread
 //               per query row; as in the one-tile kernel (lazy rescaling,
-//               packed fp32x2 math).  To fit 168 registers S is read from
-//               TMEM twice, two 32-column chunks at a time: once for the row
-//               max, once to form P.  PARTIAL tiles are masked per 32-column
-//               chunk with a warp-uniform mode (all allowed / all masked:
-//               no read, no exponential / mixed: per-element select).
+//               packed fp32x2 math).  To fit 168 registers only S columns
+//               [0,64) stay in registers after the row max; columns [64,128)
+//               are read from TMEM again when P is formed (P overwrites only
+//               columns [0,64)).  Measured faster than re-reading all of S
+//               with per-chunk mask modes.
 //
 // TMEM (512 columns): S0 [0,128), S1 [128,256), O0 [256,256+D), O1 [384,384+D);
 // P_i (bf16 pairs) is written over S_i columns [0,64) once S_i has been read.
@@ -319,31 +319,36 @@ __global__ void __launch_bounds__(384, 1)
         tc_fence_after();
         // pass 1: row max over all 128 columns; keep columns [0,64)
         uint32_t mw[4] = {0xffffffffu, 0xffffffffu, 0xffffffffu, 0xffffffffu};
-        uint32_t modes = 0u;  // all chunks unmasked
-        if (fl & part_bit) {
+        const bool part = (fl & part_bit) != 0;
+        if (part) {
           mw[0] = mw[1] = mw[2] = mw[3] = 0u;
           if (valid) row_mask_bits(mp, qi, qk, kb * 128, mw);
-          modes = chunk_modes(mw);
         }
+        float sv[64];
         float acc[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-        // pass 1 (row max): two TMEM round trips of two chunks each
+        // two TMEM round trips: chunks {0,1} (kept) then {2,3} (max only)
 #pragma unroll
         for (int half = 0; half < 2; ++half) {
-          uint32_t r[2][32];
-          tmem_ld32(tm_s + half * 64, r[0]);
-          tmem_ld32(tm_s + half * 64 + 32, r[1]);
+          uint32_t r[64];
+          tmem_ld32(tm_s + half * 64, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
+          tmem_ld32(tm_s + half * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
           tmem_wait_ld();
+          float x[64];
+          if (part) {
 #pragma unroll
-          for (int cc = 0; cc < 2; ++cc) {
-            const int c = 2 * half + cc;
-            const uint32_t mode = (modes >> (2 * c)) & 3u;
-            if (mode == 2u) continue;
-            mask_chunk_inplace(r[cc], mw[c], mode);
+            for (int e = 0; e < 64; ++e)
+              x[e] = ((mw[2 * half + (e >> 5)] >> (e & 31)) & 1u) ? __uint_as_float(r[e]) : -INFINITY;
+          } else {
 #pragma unroll
-            for (int e = 0; e < 32; e += 8)
+            for (int e = 0; e < 64; ++e) x[e] = __uint_as_float(r[e]);
+          }
 #pragma unroll
-              for (int k = 0; k < 4; ++k)
-                acc[k] = max3f(acc[k], __uint_as_float(r[cc][e + k]), __uint_as_float(r[cc][e + 4 + k]));
+          for (int e = 0; e < 64; e += 8)
+#pragma unroll
+            for (int k = 0; k < 4; ++k) acc[k] = max3f(acc[k], x[e + k], x[e + 4 + k]);
+          if (half == 0) {
+#pragma unroll
+            for (int e = 0; e < 64; ++e) sv[e] = x[e];
           }
         }
         const float m_tile = max3f(acc[0], acc[1], fmaxf(acc[2], acc[3])) * p.scale_log2;
@@ -373,49 +378,56 @@ __global__ void __launch_bounds__(384, 1)
         const uint64_t sl2 = f2_pack(p.scale_log2, p.scale_log2);
         const uint64_t negm = f2_pack(-m_use, -m_use);
         uint64_t acc2[4] = {0ull, 0ull, 0ull, 0ull};
-        // P from 32 logits x -> 16 packed bf16 pairs into TMEM columns [16 c, 16 c + 16);
-        // a chunk the whole warp masks is P = 0 without any exponential
+        // P from 32 logits x -> 16 packed bf16 pairs into TMEM columns [16 c, 16 c + 16)
         auto make_p = [&](const float (&x)[32], int c) {
           uint32_t w[16];
-          if (((modes >> (2 * c)) & 3u) == 2u) {
 #pragma unroll
-            for (int e = 0; e < 16; ++e) w[e] = 0u;
-          } else {
-#pragma unroll
-            for (int e = 0; e < 16; ++e) {
-              const uint64_t xs = f2_fma(f2_pack(x[2 * e], x[2 * e + 1]), sl2, negm);
-              uint64_t pe;
-              if (use_poly_exp(e)) {
-                pe = exp2_poly_x2(xs);
-              } else {
-                float x0, x1;
-                f2_unpack(xs, x0, x1);
-                pe = f2_pack(ex2_approx(x0), ex2_approx(x1));
-              }
-              acc2[e & 3] = f2_add(acc2[e & 3], pe);
-              float p0, p1;
-              f2_unpack(pe, p0, p1);
-              w[e] = pack_bf16x2(p0, p1);
+          for (int e = 0; e < 16; ++e) {
+            const uint64_t xs = f2_fma(f2_pack(x[2 * e], x[2 * e + 1]), sl2, negm);
+            uint64_t pe;
+            if (use_poly_exp(e)) {
+              pe = exp2_poly_x2(xs);
+            } else {
+              float x0, x1;
+              f2_unpack(xs, x0, x1);
+              pe = f2_pack(ex2_approx(x0), ex2_approx(x1));
             }
+            acc2[e & 3] = f2_add(acc2[e & 3], pe);
+            float p0, p1;
+            f2_unpack(pe, p0, p1);
+            w[e] = pack_bf16x2(p0, p1);
           }
           tmem_st16(tm_s + c * 16, w);
         };
-        // pass 2 (P): S is read again two chunks at a time; the pair {0,1} is read
-        // completely before P (columns [0,64)) overwrites it
+        {
+          float x0[32];
 #pragma unroll
-        for (int half = 0; half < 2; ++half) {
-          uint32_t r[2][32];
-          const uint32_t m0 = (modes >> (4 * half)) & 3u, m1 = (modes >> (4 * half + 2)) & 3u;
-          if (m0 != 2u) tmem_ld32(tm_s + half * 64, r[0]);
-          if (m1 != 2u) tmem_ld32(tm_s + half * 64 + 32, r[1]);
-          tmem_wait_ld();
+          for (int e = 0; e < 32; ++e) x0[e] = sv[e];
+          make_p(x0, 0);
+        }
+        // re-read chunk 2 while chunk 1 is turned into P (P only overwrites columns [0,64))
+        uint32_t r2[32], r3[32];
+        tmem_ld32(tm_s + 64, r2);
+        {
+          float x1[32];
 #pragma unroll
-          for (int cc = 0; cc < 2; ++cc) {
-            const int c = 2 * half + cc;
-            const uint32_t mode = (modes >> (2 * c)) & 3u;
-            if (mode != 2u) mask_chunk_inplace(r[cc], mw[c], mode);
-            make_p(*reinterpret_cast<const float(*)[32]>(&r[cc][0]), c);
+          for (int e = 0; e < 32; ++e) x1[e] = sv[32 + e];
+          make_p(x1, 1);
+        }
+        tmem_ld32(tm_s + 96, r3);
+        tmem_wait_ld();
+#pragma unroll
+        for (int c = 2; c < 4; ++c) {
+          const uint32_t (&r)[32] = c == 2 ? r2 : r3;
+          float x[32];
+          if (part) {
+#pragma unroll
+            for (int e = 0; e < 32; ++e) x[e] = ((mw[c] >> e) & 1u) ? __uint_as_float(r[e]) : -INFINITY;
+          } else {
+#pragma unroll
+            for (int e = 0; e < 32; ++e) x[e] = __uint_as_float(r[e]);
           }
+          make_p(x, c);
         }
         const uint64_t s01 = f2_add(f2_add(acc2[0], acc2[1]), f2_add(acc2[2], acc2[3]));
         float s0, s1;
