@@ -147,10 +147,6 @@ struct BwdBars {
   int abort;
 };
 
-__device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
-}
-
 // ---------------------------------------------------------------------------
 // 2. dK, dV: key-major walk of the CSC
 // ---------------------------------------------------------------------------

@@ -17,15 +17,17 @@
 //   warp 1      TMEM allocator, single-thread tcgen05.mma issuer.  Per union
 //               column u and tile i: first O_i += P_i(u') V(u') for the tile's
 //               pending column u' < u, then S_i(u) = Q_i K(u)^T.  The order
-//               PV0, S0, PV1, S1 gives each softmax warpgroup the other
-//               tile's two MMAs (1024 tensor cycles) to turn S into P.
-//   warps 4-7   softmax warpgroup of tile 0, warps 8-11 of tile 1: one thread
-//               per query row; as in the one-tile kernel (lazy rescaling,
-//               packed fp32x2 math).  To fit 168 registers only S columns
-//               [0,64) stay in registers after the row max; columns [64,128)
-//               are read from TMEM again when P is formed (P overwrites only
-//               columns [0,64)).  Measured faster than re-reading all of S
-//               with per-chunk mask modes.
+//               PV0, S0, PV1, S1 gives the softmax the other tile's two MMAs
+//               (1024 tensor cycles) to turn S_i into P_i.
+//   warps 4-11  softmax, both warpgroups on every S tile in turn (S0(u),
+//               S1(u), S0(u+1), ...): warpgroup wg takes key columns
+//               [64 wg, 64 wg + 64), one thread per query row; the two warps
+//               on the same TMEM lane quarter exchange row maxima through
+//               shared memory.  Lazy rescaling, packed fp32x2 math.  The MUFU
+//               (16 exponentials per clock and SM) needs all of the 1024
+//               cycles to exponentiate one 128x128 tile, so one warp per SMSP
+//               and tile left it idle during every TMEM round trip; two warps
+//               per SMSP on the same tile overlap those waits.
 //
 // TMEM (512 columns): S0 [0,128), S1 [128,256), O0 [256,256+D), O1 [384,384+D);
 // P_i (bf16 pairs) is written over S_i columns [0,64) once S_i has been read.
@@ -78,7 +80,8 @@ struct FwdPairCfg {
   static constexpr int SMEM_K = 2 * TILE_BYTES;
   static constexpr int SMEM_V = SMEM_K + K_SLOTS * TILE_BYTES;
   static constexpr int SMEM_BAR = SMEM_V + V_SLOTS * TILE_BYTES;
-  static constexpr int SMEM_BYTES = SMEM_BAR + 512 + 1024;
+  static constexpr int SMEM_X = SMEM_BAR + 256;        // float[2][128] row exchange
+  static constexpr int SMEM_BYTES = SMEM_X + 1024 + 1024;
   static constexpr uint32_t TM_S = 0, TM_O = 256;
 };
 
@@ -89,6 +92,15 @@ struct PairBars {
   uint32_t tmem_base;
   int abort;
 };
+static_assert(sizeof(PairBars) <= 256, "barriers overlap the row exchange buffer");
+
+// Exponential pairs computed on the FMA pipe (exp2_poly_x2) instead of the
+// MUFU: bit e of the mask selects pair e of every 16-pair (32-key) chunk.
+// The MUFU issues 16 exponentials per clock and SM -- exactly what the tensor
+// core's 128x128x128 S and PV tiles need in the same time -- so a share on
+// the FMA pipe gives it headroom.
+constexpr uint32_t kPairPolyMask = 0u;
+__host__ __device__ constexpr bool use_poly_pair(int e) { return ((kPairPolyMask >> e) & 1u) != 0u; }
 
 template <int D>
 __global__ void __launch_bounds__(384, 1)
@@ -118,9 +130,9 @@ __global__ void __launch_bounds__(384, 1)
       mbar_init(&bars->v_full[i], 1);
       mbar_init(&bars->v_empty[i], 1);
       mbar_init(&bars->s_full[i], 1);
-      mbar_init(&bars->p_full[i], 128);
+      mbar_init(&bars->p_full[i], 256);
       mbar_init(&bars->o_full[i], 1);
-      mbar_init(&bars->o_empty[i], 128);
+      mbar_init(&bars->o_empty[i], 256);
     }
     fence_barrier_init();
   }
@@ -273,15 +285,31 @@ __global__ void __launch_bounds__(384, 1)
       mbar_wait_drain(&bars->mma_done, 0);
     }
   } else if (warp >= 4) {
-    // ------------------------------------------------------------ softmax WGs
-    const int ti = (warp - 4) >> 2;            // which query tile of the pair
-    const int quarter = warp & 3;              // TMEM lane quarter
+    // ------------------------------------------------------------ softmax
+    // Both warpgroups work on every S tile: warpgroup wg owns its key
+    // columns [64 wg, 64 wg + 64), warp (wg, quarter) the 32 rows of TMEM
+    // lane quarter `quarter`.  The two warps sharing a quarter (same rows,
+    // same SMSP) exchange partial row maxima -- and at the end row sums --
+    // through shared memory under a 64-thread named barrier, so both apply
+    // the same running maximum m.  Two warps per SMSP keep the MUFU busy
+    // while one of them waits on TMEM or the exchange.
+    const int wg = (warp - 4) >> 2;
+    const int quarter = warp & 3;
     const int row = quarter * 32 + lane;
     const uint32_t lane_addr = static_cast<uint32_t>(quarter * 32) << 16;
-    const uint32_t tm_s = tmem + lane_addr + C::TM_S + ti * 128;
-    const uint32_t tm_o = tmem + lane_addr + C::TM_O + ti * 128;
-    const uint8_t in_bit = ti == 0 ? kPairIn0 : kPairIn1;
-    const uint8_t part_bit = ti == 0 ? kPairPart0 : kPairPart1;
+    const int col0 = wg * 64;
+    float* xchg = reinterpret_cast<float*>(smem + C::SMEM_X);
+    volatile float* x_mine = xchg + wg * 128 + row;
+    volatile float* x_peer = xchg + (1 - wg) * 128 + row;
+    const int bar_id = 1 + quarter;
+    // write v, read the peer's: the first barrier guarantees the peer has read
+    // the previous value, the second that it has written this one
+    auto exchange = [&](float v) {
+      named_bar_sync(bar_id, 64);
+      *x_mine = v;
+      named_bar_sync(bar_id, 64);
+      return *x_peer;
+    };
     constexpr float kRescaleThreshold = 8.0f;
     FwdParams mp{};
     mp.f = p.f;
@@ -290,20 +318,24 @@ __global__ void __launch_bounds__(384, 1)
     mp.sink = p.sink;
     mp.hd = p.hd;
     mp.cd = p.cd;
-    uint32_t g = 0, icnt = 0;
+    uint32_t g[2] = {0u, 0u}, icnt[2] = {0u, 0u};
     for (int item = blockIdx.x; item < p.items; item += gridDim.x) {
       const int bh = item / p.np;
       const int pr = p.pair_order ? p.pair_order[item - bh * p.np] : item - bh * p.np;
-      const int t = 2 * pr + ti;
-      if (t >= p.nt) continue;  // odd tail: this pair has one tile
       const int b = bh / p.heads, h = bh - b * p.heads;
-      const int a = t * 128 + row;
-      const bool valid = a < p.n;
-      const int qi = valid ? a / p.s : 0;
-      const int qk = valid ? a - qi * p.s : 0;
+      const bool two = 2 * pr + 1 < p.nt;
       const int u0 = p.pair_ptr[pr], u1 = p.pair_ptr[pr + 1];
-      float m = -INFINITY, l = 0.f;
-      bool first = true;
+      float m[2] = {-INFINITY, -INFINITY}, l[2] = {0.f, 0.f};
+      bool first[2] = {true, true};
+      int qi[2], qk[2];
+      bool valid[2];
+#pragma unroll
+      for (int ti = 0; ti < 2; ++ti) {
+        const int a = (2 * pr + ti) * 128 + row;
+        valid[ti] = a < p.n;
+        qi[ti] = valid[ti] ? a / p.s : 0;
+        qk[ti] = valid[ti] ? a - qi[ti] * p.s : 0;
+      }
       uint8_t fl_next = p.pair_flag[u0];
       int kb_next = p.pair_col[u0];
       for (int u = u0; u < u1; ++u) {
@@ -313,161 +345,153 @@ __global__ void __launch_bounds__(384, 1)
           fl_next = p.pair_flag[u + 1];
           kb_next = p.pair_col[u + 1];
         }
-        if (!(fl & in_bit)) continue;
-        mbar_wait(&bars->s_full[ti], g & 1, abort_flag);
-        __syncwarp();
-        tc_fence_after();
-        // pass 1: row max over all 128 columns; keep columns [0,64)
-        uint32_t mw[4] = {0xffffffffu, 0xffffffffu, 0xffffffffu, 0xffffffffu};
-        const bool part = (fl & part_bit) != 0;
-        if (part) {
-          mw[0] = mw[1] = mw[2] = mw[3] = 0u;
-          if (valid) row_mask_bits(mp, qi, qk, kb * 128, mw);
-        }
-        float sv[64];
-        float acc[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-        // two TMEM round trips: chunks {0,1} (kept) then {2,3} (max only)
 #pragma unroll
-        for (int half = 0; half < 2; ++half) {
+        for (int ti = 0; ti < 2; ++ti) {
+          if (!(fl & (ti == 0 ? kPairIn0 : kPairIn1))) continue;
+          mbar_wait(&bars->s_full[ti], g[ti] & 1, abort_flag);
+          __syncwarp();
+          tc_fence_after();
+          const uint32_t tm_s = tmem + lane_addr + C::TM_S + ti * 128;
           uint32_t r[64];
-          tmem_ld32(tm_s + half * 64, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
-          tmem_ld32(tm_s + half * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
-          tmem_wait_ld();
-          float x[64];
+          tmem_ld32(tm_s + col0, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
+          tmem_ld32(tm_s + col0 + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
+          // the mask bits of a PARTIAL tile are computed while the load is in flight
+          const bool part = (fl & (ti == 0 ? kPairPart0 : kPairPart1)) != 0;
+          uint32_t mw[4] = {0xffffffffu, 0xffffffffu, 0xffffffffu, 0xffffffffu};
+          if (part) {
+            mw[0] = mw[1] = mw[2] = mw[3] = 0u;
+            if (valid[ti]) row_mask_bits(mp, qi[ti], qk[ti], kb * 128 + col0, mw);
+          }
+          uint32_t live = 3u;  // 32-key chunks with an allowed key in some lane of the warp
+          uint32_t mixed = 0u;  // chunks that need the per-element select
           if (part) {
 #pragma unroll
-            for (int e = 0; e < 64; ++e)
-              x[e] = ((mw[2 * half + (e >> 5)] >> (e & 31)) & 1u) ? __uint_as_float(r[e]) : -INFINITY;
-          } else {
-#pragma unroll
-            for (int e = 0; e < 64; ++e) x[e] = __uint_as_float(r[e]);
+            for (int c = 0; c < 2; ++c) {
+              if (!__any_sync(0xffffffffu, mw[c] != 0u)) live &= ~(1u << c);
+              else if (!__all_sync(0xffffffffu, mw[c] == 0xffffffffu)) mixed |= 1u << c;
+            }
           }
+          tmem_wait_ld();
+          float acc[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-          for (int e = 0; e < 64; e += 8)
+          for (int c = 0; c < 2; ++c) {
+            if (mixed & (1u << c)) {
 #pragma unroll
-            for (int k = 0; k < 4; ++k) acc[k] = max3f(acc[k], x[e + k], x[e + 4 + k]);
-          if (half == 0) {
+              for (int e = 0; e < 32; ++e)
+                if (!((mw[c] >> e) & 1u)) r[32 * c + e] = 0xff800000u;  // -inf
+            }
+            if (live & (1u << c)) {
 #pragma unroll
-            for (int e = 0; e < 64; ++e) sv[e] = x[e];
+              for (int e = 32 * c; e < 32 * c + 32; e += 8)
+#pragma unroll
+                for (int k = 0; k < 4; ++k) acc[k] = max3f(acc[k], __uint_as_float(r[e + k]), __uint_as_float(r[e + 4 + k]));
+            }
           }
-        }
-        const float m_tile = max3f(acc[0], acc[1], fmaxf(acc[2], acc[3])) * p.scale_log2;
-        const bool grow = m_tile > m + kRescaleThreshold;
-        if (!first) {
-          if (__any_sync(0xffffffffu, grow)) {
-            // O_i already holds every earlier PV (covered by the S commit).
-            const float factor = grow ? ex2_approx(m - m_tile) : 1.0f;
+          const float mloc = max3f(acc[0], acc[1], fmaxf(acc[2], acc[3]));
+          const float m_tile = fmaxf(mloc, exchange(mloc)) * p.scale_log2;
+          // lazy rescaling: m moves only when the tile's maximum exceeds it by
+          // more than the threshold (P stays below 2^8)
+          const bool grow = m_tile > m[ti] + kRescaleThreshold;
+          const bool resc = !first[ti] && __any_sync(0xffffffffu, grow);
+          const float factor = (grow && !first[ti]) ? ex2_approx(m[ti] - m_tile) : 1.0f;
+          if (grow) {
+            l[ti] *= factor;
+            m[ti] = m_tile;
+          }
+          const float m_use = (m[ti] == -INFINITY) ? 0.f : m[ti];
+          const uint64_t sl2 = f2_pack(p.scale_log2, p.scale_log2);
+          const uint64_t negm = f2_pack(-m_use, -m_use);
+          uint64_t acc2[2] = {0ull, 0ull};
 #pragma unroll
-            for (int c = 0; c < D / 32; ++c) {
-              uint32_t r[32];
-              tmem_ld32(tm_o + c * 32, r);
+          for (int c = 0; c < 2; ++c) {
+            uint32_t w[16];
+            if (!(live & (1u << c))) {
+#pragma unroll
+              for (int e = 0; e < 16; ++e) w[e] = 0u;
+              tmem_st16(tm_s + wg * 32 + c * 16, w);
+              continue;
+            }
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+              const int k2 = 32 * c + 2 * e;
+              const uint64_t xs = f2_fma(f2_pack(__uint_as_float(r[k2]), __uint_as_float(r[k2 + 1])), sl2, negm);
+              uint64_t pe;
+              if (use_poly_pair(e)) {
+                pe = exp2_poly_x2(xs);
+              } else {
+                float x0, x1;
+                f2_unpack(xs, x0, x1);
+                pe = f2_pack(ex2_approx(x0), ex2_approx(x1));
+              }
+              acc2[e & 1] = f2_add(acc2[e & 1], pe);
+              float p0, p1;
+              f2_unpack(pe, p0, p1);
+              w[e] = pack_bf16x2(p0, p1);
+            }
+            // P (bf16 pairs) of keys [col0 + 32 c, +32) -> TMEM columns (col0 + 32 c) / 2
+            tmem_st16(tm_s + wg * 32 + c * 16, w);
+          }
+          const uint64_t s01 = f2_add(acc2[0], acc2[1]);
+          float s0, s1;
+          f2_unpack(s01, s0, s1);
+          l[ti] += s0 + s1;
+          if (resc) {
+            // O_i holds every earlier PV (the S commit covers them); this
+            // warp rescales its half of the output columns
+            const uint32_t tm_o = tmem + lane_addr + C::TM_O + ti * 128 + wg * (D / 2);
+#pragma unroll
+            for (int c = 0; c < D / 64; ++c) {
+              uint32_t ro[32];
+              tmem_ld32(tm_o + c * 32, ro);
               tmem_wait_ld();
 #pragma unroll
-              for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * factor);
-              tmem_st32(tm_o + c * 32, r);
-            }
-            if (grow) {
-              l *= factor;
-              m = m_tile;
+              for (int e = 0; e < 32; ++e) ro[e] = __float_as_uint(__uint_as_float(ro[e]) * factor);
+              tmem_st32(tm_o + c * 32, ro);
             }
           }
-        } else if (grow) {
-          m = m_tile;
+          tmem_wait_st();
+          tc_fence_before();
+          mbar_arrive(&bars->p_full[ti]);
+          first[ti] = false;
+          ++g[ti];
         }
-        const float m_use = (m == -INFINITY) ? 0.f : m;
-        const uint64_t sl2 = f2_pack(p.scale_log2, p.scale_log2);
-        const uint64_t negm = f2_pack(-m_use, -m_use);
-        uint64_t acc2[4] = {0ull, 0ull, 0ull, 0ull};
-        // P from 32 logits x -> 16 packed bf16 pairs into TMEM columns [16 c, 16 c + 16)
-        auto make_p = [&](const float (&x)[32], int c) {
-          uint32_t w[16];
-#pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            const uint64_t xs = f2_fma(f2_pack(x[2 * e], x[2 * e + 1]), sl2, negm);
-            uint64_t pe;
-            if (use_poly_exp(e)) {
-              pe = exp2_poly_x2(xs);
-            } else {
-              float x0, x1;
-              f2_unpack(xs, x0, x1);
-              pe = f2_pack(ex2_approx(x0), ex2_approx(x1));
-            }
-            acc2[e & 3] = f2_add(acc2[e & 3], pe);
-            float p0, p1;
-            f2_unpack(pe, p0, p1);
-            w[e] = pack_bf16x2(p0, p1);
-          }
-          tmem_st16(tm_s + c * 16, w);
-        };
-        {
-          float x0[32];
-#pragma unroll
-          for (int e = 0; e < 32; ++e) x0[e] = sv[e];
-          make_p(x0, 0);
-        }
-        // re-read chunk 2 while chunk 1 is turned into P (P only overwrites columns [0,64))
-        uint32_t r2[32], r3[32];
-        tmem_ld32(tm_s + 64, r2);
-        {
-          float x1[32];
-#pragma unroll
-          for (int e = 0; e < 32; ++e) x1[e] = sv[32 + e];
-          make_p(x1, 1);
-        }
-        tmem_ld32(tm_s + 96, r3);
-        tmem_wait_ld();
-#pragma unroll
-        for (int c = 2; c < 4; ++c) {
-          const uint32_t (&r)[32] = c == 2 ? r2 : r3;
-          float x[32];
-          if (part) {
-#pragma unroll
-            for (int e = 0; e < 32; ++e) x[e] = ((mw[c] >> e) & 1u) ? __uint_as_float(r[e]) : -INFINITY;
-          } else {
-#pragma unroll
-            for (int e = 0; e < 32; ++e) x[e] = __uint_as_float(r[e]);
-          }
-          make_p(x, c);
-        }
-        const uint64_t s01 = f2_add(f2_add(acc2[0], acc2[1]), f2_add(acc2[2], acc2[3]));
-        float s0, s1;
-        f2_unpack(s01, s0, s1);
-        l += s0 + s1;
-        tmem_wait_st();
-        tc_fence_before();
-        mbar_arrive(&bars->p_full[ti]);
-        first = false;
-        ++g;
       }
       // -------------------------------------------------------- epilogue
-      mbar_wait(&bars->o_full[ti], icnt & 1, abort_flag);
-      __syncwarp();
-      tc_fence_after();
-      const float inv_l = l > 0.f ? 1.0f / l : 0.f;
-      __nv_bfloat16* orow = p.o + static_cast<int64_t>(b) * p.o_sb + static_cast<int64_t>(h) * p.o_sh +
-                            static_cast<int64_t>(valid ? a : 0) * p.o_sn;
 #pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
-        uint32_t r[32];
-        tmem_ld32(tm_o + c * 32, r);
-        tmem_wait_ld();
-        if (valid) {
-          uint32_t pk[16];
+      for (int ti = 0; ti < 2; ++ti) {
+        if (ti == 1 && !two) break;  // odd tail: this pair has one tile
+        mbar_wait(&bars->o_full[ti], icnt[ti] & 1, abort_flag);
+        __syncwarp();
+        tc_fence_after();
+        const float lt = l[ti] + exchange(l[ti]);
+        const float inv_l = lt > 0.f ? 1.0f / lt : 0.f;
+        const int a = (2 * pr + ti) * 128 + row;
+        __nv_bfloat16* orow = p.o + static_cast<int64_t>(b) * p.o_sb + static_cast<int64_t>(h) * p.o_sh +
+                              static_cast<int64_t>(valid[ti] ? a : 0) * p.o_sn + wg * (D / 2);
+        const uint32_t tm_o = tmem + lane_addr + C::TM_O + ti * 128 + wg * (D / 2);
 #pragma unroll
-          for (int e = 0; e < 16; ++e)
-            pk[e] = pack_bf16x2(__uint_as_float(r[2 * e]) * inv_l, __uint_as_float(r[2 * e + 1]) * inv_l);
-          uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
+        for (int c = 0; c < D / 64; ++c) {
+          uint32_t ro[32];
+          tmem_ld32(tm_o + c * 32, ro);
+          tmem_wait_ld();
+          if (valid[ti]) {
+            uint32_t pk[16];
 #pragma unroll
-          for (int v = 0; v < 4; ++v) dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+            for (int e = 0; e < 16; ++e)
+              pk[e] = pack_bf16x2(__uint_as_float(ro[2 * e]) * inv_l, __uint_as_float(ro[2 * e + 1]) * inv_l);
+            uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
+#pragma unroll
+            for (int v = 0; v < 4; ++v) dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+          }
         }
+        tc_fence_before();
+        mbar_arrive(&bars->o_empty[ti]);
+        if (wg == 0 && valid[ti]) {
+          const float lse = lt > 0.f ? (m[ti] + log2f(lt)) * 0.69314718055994531f : -INFINITY;
+          p.lse[(static_cast<int64_t>(b) * p.heads + h) * p.n + a] = lse;
+        }
+        ++icnt[ti];
       }
-      tc_fence_before();
-      mbar_arrive(&bars->o_empty[ti]);
-      if (valid) {
-        const float lse = l > 0.f ? (m + log2f(l)) * 0.69314718055994531f : -INFINITY;
-        p.lse[(static_cast<int64_t>(b) * p.heads + h) * p.n + a] = lse;
-      }
-      ++icnt;
     }
   }
 

@@ -345,6 +345,12 @@ __device__ __forceinline__ uint64_t exp2_poly_x2(uint64_t x) {
                  __int_as_float(__float_as_int(q1) + (j1 << 23)));
 }
 
+// Named barrier over the first `nthreads` threads that reach barrier `id`
+// (ids 1..15; 0 is __syncthreads).
+__device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   uint32_t r;
   asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
