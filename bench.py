@@ -432,7 +432,7 @@ def run_sweep(args, dev, stream, peak):
 
 def fwd_kernel_name():
     single = os.environ.get("RADIAL_FWD_KERNEL") == "single"
-    return "radial_fwd_kernel<128,1>" if single else "radial_fwd_pair_kernel<128>"
+    return "radial_fwd_kernel<128>" if single else "radial_fwd_pair_kernel<128>"
 
 
 def kernel_sha():

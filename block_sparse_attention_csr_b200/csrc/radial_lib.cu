@@ -495,16 +495,6 @@ radial_status check_desc(const radial_csr* c, const radial_desc* d) {
   return RADIAL_OK;
 }
 
-// RADIAL_FWD_SOFTMAX=classic selects the one-MUFU-per-element softmax loop
-// (kept for comparison); the default is the packed / partly polynomial one.
-bool fwd_classic_softmax() {
-  static const bool classic = [] {
-    const char* e = std::getenv("RADIAL_FWD_SOFTMAX");
-    return e && std::strcmp(e, "classic") == 0;
-  }();
-  return classic;
-}
-
 float softmax_scale(const radial_desc* d) {
   return d->scale > 0.f ? d->scale : 1.0f / std::sqrt(static_cast<float>(d->head_dim));
 }
@@ -598,13 +588,8 @@ radial_status launch_fwd(const radial_csr* c, const radial_desc* d, const void* 
   p.scale_log2 = softmax_scale(d) * 1.4426950408889634f;
   const int smem = FwdCfg<D>::SMEM_BYTES;
   const int grid = p.items < sm_count() ? p.items : sm_count();
-  if (fwd_classic_softmax()) {
-    RADIAL_CUDA(cudaFuncSetAttribute(radial_fwd_kernel<D, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
-    radial_fwd_kernel<D, false><<<grid, 192, smem, st>>>(mq, mk, mv, p);
-  } else {
-    RADIAL_CUDA(cudaFuncSetAttribute(radial_fwd_kernel<D, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
-    radial_fwd_kernel<D, true><<<grid, 192, smem, st>>>(mq, mk, mv, p);
-  }
+  RADIAL_CUDA(cudaFuncSetAttribute(radial_fwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
+  radial_fwd_kernel<D><<<grid, 384, smem, st>>>(mq, mk, mv, p);
   RADIAL_LAUNCHED();
   return RADIAL_OK;
 }
