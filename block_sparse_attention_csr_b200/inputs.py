@@ -105,3 +105,22 @@ def draw_fp32(wl: Workload, backward=None):
             x.mul_(wl.value_scale)
         out.append(x)
     return tuple(out)
+
+
+def draw_lora_layer(batch, heads, head_dim, frames, tokens_per_frame, rank, seed, device="cpu"):
+    """Seeded synthetic inputs of one LoRA-adapted attention layer step, all
+    bf16: activations x and upstream gradient dy [B, N, C] ~ N(0, 1); frozen
+    projections W_p [C, C] ~ N(0, 1/C) (unit-variance outputs); adapters
+    A_p [r, C] ~ N(0, 1/C) and B_p [C, r] ~ N(0, 1/r) for p in q, k, v, o.
+    (Fine-tuning starts from B = 0; random B exercises the adapter path.)
+    Drawn on the CPU in the order x, dy, then W, A, B per projection."""
+    C = heads * head_dim
+    N = frames * tokens_per_frame
+    g = torch.Generator(device="cpu")
+    g.manual_seed(seed)
+    out = {"x": torch.randn(batch, N, C, generator=g), "dy": torch.randn(batch, N, C, generator=g)}
+    for p in ("q", "k", "v", "o"):
+        out["W_" + p] = torch.randn(C, C, generator=g) / C ** 0.5
+        out["A_" + p] = torch.randn(rank, C, generator=g) / C ** 0.5
+        out["B_" + p] = torch.randn(C, rank, generator=g) / rank ** 0.5
+    return {k: v.to(torch.bfloat16).to(device) for k, v in out.items()}

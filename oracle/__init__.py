@@ -28,6 +28,7 @@ Modules:
 
 * :mod:`oracle.mask`      -- the token-level mask, its block-level CSR.
 * :mod:`oracle.attention` -- masked softmax attention forward and backward.
+* :mod:`oracle.lora`      -- LoRA-wrapped Q/K/V/O projections around it ([review] §4.3).
 
 Parity status per function is stated in each module header.
 """
