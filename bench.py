@@ -308,6 +308,9 @@ def run_ours(args, rank, world, local_rank):
     if rank == 0 and args.sweep:
         extra["sweep"] = run_sweep(args, dev, stream, peak)
 
+    if rank == 0 and args.lora:
+        extra["lora_layer"] = run_lora_layer(wl, csr, dev, stream, args.lora_rank)
+
     # ---- end to end through the public API with host buffers
     e2e = None
     if rank == 0 and not args.quick:
@@ -430,6 +433,42 @@ def run_sweep(args, dev, stream, peak):
     return out
 
 
+def run_lora_layer(wl, csr, dev, stream, r):
+    """One LoRA-adapted attention layer step (forward + backward: dx and the
+    adapter gradients) at the workload's shape, hidden size heads*head_dim,
+    adapter rank r: projections in cuBLAS, attention in the library."""
+    import numpy as np
+    import torch
+    from block_sparse_attention_csr_b200 import inputs as I
+    from block_sparse_attention_csr_b200.lora import RadialLoRALayer
+
+    t = I.draw_lora_layer(wl.batch, wl.heads, wl.head_dim, wl.frames, wl.tokens_per_frame, r, wl.seed + 100,
+                          device=dev)
+    layer = RadialLoRALayer(csr, wl.heads, {k: v for k, v in t.items() if k.startswith("W_")},
+                            {k: v for k, v in t.items() if k[:2] in ("A_", "B_")}, 1.0)
+
+    def lstep():
+        y, ctx = layer.forward(t["x"])
+        return layer.backward(ctx, t["dy"])
+
+    for _ in range(2):
+        lstep()
+    e = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(3)]
+    for a, b in e:
+        a.record(stream)
+        lstep()
+        b.record(stream)
+    torch.cuda.synchronize(dev)
+    ms = float(np.mean([a.elapsed_time(b) for a, b in e]))
+    C, n = wl.heads * wl.head_dim, wl.batch * wl.n
+    # per projection: forward 2nC^2 + 4nCr, backward (dx, dA, dB) 2nC^2 + 8nCr
+    proj_flops = 4 * (4 * n * C * C + 12 * n * C * r)
+    del t, layer
+    torch.cuda.empty_cache()
+    return {"rank": r, "hidden": C, "ms_per_step": ms, "projection_gemm_tflop": proj_flops / 1e12,
+            "path": "4 LoRA projections (cuBLAS GEMMs) + radial_attn_fwd/bwd (this library), forward + backward"}
+
+
 def fwd_kernel_name():
     single = os.environ.get("RADIAL_FWD_KERNEL") == "single"
     return "radial_fwd_kernel<128>" if single else "radial_fwd_pair_kernel<128>"
@@ -506,6 +545,8 @@ def main():
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--ref-rows", type=int, default=512)
     ap.add_argument("--sweep", action="store_true", help="add the frame-count scaling sweep (radial vs dense)")
+    ap.add_argument("--lora", action="store_true", help="add one LoRA-adapted attention layer step (fwd+bwd)")
+    ap.add_argument("--lora-rank", type=int, default=64)
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         args.warmup = 3
