@@ -47,10 +47,6 @@ __device__ __forceinline__ long long period_of(const int32_t* cd, int s, int d) 
   return ((1LL << r) + s - 1) / s;
 }
 
-__device__ __forceinline__ int band_of(int d) {  // floor(log2(max(d,1)))
-  return 31 - __clz(d > 1 ? d : 1);
-}
-
 // Segment pair test.  Query positions [k0,k1] of frame i against key positions
 // [l0,l1] of frame j.  Sets any / all for "some pair allowed" / "every pair".
 __device__ __forceinline__ void segment_pair(const MaskGeom& g, int i, int k0, int k1, int j, int l0,
