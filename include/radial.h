@@ -213,9 +213,10 @@ radial_status radial_device_status(void* stream);
  * as designed. */
 radial_status radial_selftest_bounded_wait(uint32_t limit_ms, void* stream);
 
-/* Self-test of the polynomial base-2 exponential the forward softmax runs on
- * the FMA pipe for part of its elements: y[i] = 2^x[i] for n device floats
- * (inputs below -125 give about 2^-125).  Asynchronous. */
+/* Self-test of the polynomial base-2 exponential that the forward softmax
+ * can run on the FMA pipe for part of its elements (a compile-time switch,
+ * off by default: measured no faster than the MUFU alone): y[i] = 2^x[i] for
+ * n device floats (inputs below -125 give about 2^-125).  Asynchronous. */
 radial_status radial_selftest_exp2(const float* x, float* y, int32_t n, void* stream);
 
 /* Static text for a status code. */
