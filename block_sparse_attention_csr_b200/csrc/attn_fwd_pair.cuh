@@ -10,7 +10,7 @@
 // shifted by 128 tokens); a key tile only one of them needs is computed for
 // that tile alone.
 //
-// Warp roles (384 threads, 168 registers each):
+// Warp roles (384 threads; at most 168 registers each, 148 used):
 //   warp 0      TMA producer: Q0, Q1 once per item; K and V through
 //               separate 3-slot / 2-slot rings, K one union column ahead of V.
 //   warps 2-3   idle (keep the softmax warps on warpgroup boundaries).

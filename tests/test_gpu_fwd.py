@@ -144,3 +144,18 @@ def test_hunyuan720p_sampled_rows():
 @pytest.mark.slow
 def test_hunyuan720p_4x_sampled_rows():
     _sampled_check("hunyuan720p_4x", int(os.environ.get("RADIAL_4X_ROWS", "4096")))
+
+
+def test_one_tile_kernel_all_rows():
+    """The alternate forward (one query tile per CTA, double-buffered S),
+    selected per process by RADIAL_FWD_KERNEL=single: the all-row parity
+    cases above, run in a child process with that variable set."""
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    env = dict(os.environ, RADIAL_FWD_KERNEL="single")
+    r = subprocess.run([sys.executable, "-m", "pytest", os.path.join(root, "tests", "test_gpu_fwd.py"), "-q",
+                        "-p", "no:cacheprovider", "-m", "gpu",
+                        "-k", "test_tiny_config_all_rows or test_small_all_rows or test_strided_layout"],
+                       cwd=root, env=env, capture_output=True, text=True, timeout=1200)
+    assert r.returncode == 0, r.stdout[-3000:] + r.stderr[-2000:]
