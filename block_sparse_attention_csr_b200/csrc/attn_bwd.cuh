@@ -143,9 +143,11 @@ struct BwdBars {
   uint64_t fix_full, fix_empty, acc_empty, mma_done;
   uint64_t s_full, s_free, ew_full[2], mma2_done[2];
   uint64_t st_full[2], st_empty[2];
+  uint64_t dp_full, p_ready[2], ds_ready[2];  // dK/dV kernel: S^T and dP^T halves of the handoff
   uint32_t tmem_base;
   int abort;
 };
+static_assert(sizeof(BwdBars) <= 256, "barrier area");
 
 // ---------------------------------------------------------------------------
 // 2. dK, dV: key-major walk of the CSC
@@ -155,6 +157,13 @@ struct BwdBars {
 // (query columns [0,64) and [64,128) of each tile).  Warpgroup wg writes its
 // bf16 P^T over S^T columns [64 wg, 64 wg + 32) and its dS^T over dP^T columns
 // [64 wg, 64 wg + 32), i.e. over values it has already read.
+// The elementwise work of a query tile runs in two passes, each released to
+// the MMA thread on its own barrier: P^T (needs only S^T) and then dS^T (needs
+// dP^T and the P^T values kept in registers).  The MMA stream per tile g is
+// dV(g), S^T(g+1), dK(g), dP^T(g+1): dV(g) and the next S^T run while the
+// elementwise warps form dS^T(g), and dK(g) and the next dP^T while they form
+// P^T(g+1).  Each new S^T / dP^T follows, in the same in-order MMA stream,
+// the MMA that reads the P^T / dS^T it overwrites.
 template <int D>
 __global__ void __launch_bounds__(384, 1)
     radial_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -181,7 +190,10 @@ __global__ void __launch_bounds__(384, 1)
     mbar_init(&bars->mma_done, 1);
     mbar_init(&bars->s_full, 1);
     mbar_init(&bars->s_free, 128);
+    mbar_init(&bars->dp_full, 1);
     for (int b = 0; b < 2; ++b) {
+      mbar_init(&bars->p_ready[b], 256);
+      mbar_init(&bars->ds_ready[b], 256);
       mbar_init(&bars->ew_full[b], 256);
       mbar_init(&bars->mma2_done[b], 1);
       mbar_init(&bars->st_full[b], 1);
@@ -246,32 +258,47 @@ __global__ void __launch_bounds__(384, 1)
         const uint32_t n_tiles = static_cast<uint32_t>(p.col_ptr[u + 1] - p.col_ptr[u]);
         mbar_wait(&bars->fix_full, item_i & 1, abort_flag);
         tc_fence_after();
-        for (uint32_t j = 0; j < n_tiles; ++j) {
-          const uint32_t g = it + j, st = g % C::STAGES;
+        // S^T(g) = K Q_g^T and dP^T(g) = V dO_g^T (Q, dO of stage g as K-major B)
+        auto issue_s = [&](uint32_t g) {
+          const uint32_t st = g % C::STAGES;
           mbar_wait(&bars->st_full[st], (g / C::STAGES) & 1, abort_flag);
           tc_fence_after();
-          // S^T / dP^T overwrite the columns where P^T / dS^T of tile g-1 are read
-          // by its dV / dK MMAs, issued just before in the same MMA stream.
-          const uint64_t qk = dQk + st * 2 * kTile, ok = qk + kTile;
+          const uint64_t qk = dQk + st * 2 * kTile;
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
             const uint64_t off = static_cast<uint64_t>(((kk >> 2) * 16384 + (kk & 3) * 32) >> 4);
             mma_ss(tmem + TM_S, dK + off, qk + off, idesc_s, kk > 0 ? 1u : 0u);
           }
+          mma_commit(&bars->s_full);
+        };
+        auto issue_dp = [&](uint32_t g) {
+          const uint32_t st = g % C::STAGES;
+          const uint64_t ok = dQk + st * 2 * kTile + kTile;
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
             const uint64_t off = static_cast<uint64_t>(((kk >> 2) * 16384 + (kk & 3) * 32) >> 4);
             mma_ss(tmem + TM_DP, dV + off, ok + off, idesc_s, kk > 0 ? 1u : 0u);
           }
-          mma_commit(&bars->s_full);
-          mbar_wait(&bars->ew_full[g & 1], (g >> 1) & 1, abort_flag);
+          mma_commit(&bars->dp_full);
+        };
+        issue_s(it);
+        issue_dp(it);
+        for (uint32_t j = 0; j < n_tiles; ++j) {
+          const uint32_t g = it + j, st = g % C::STAGES;
+          const uint64_t qmn = dQmn + st * 2 * kTile, omn = qmn + kTile;
+          // dV(g) += P^T(g) dO_g, once the elementwise warps have written P^T(g)
+          mbar_wait(&bars->p_ready[g & 1], (g >> 1) & 1, abort_flag);
           if (j == 0 && item_i > 0) mbar_wait(&bars->acc_empty, (item_i - 1) & 1, abort_flag);
           tc_fence_after();
-          const uint64_t qmn = dQmn + st * 2 * kTile, omn = qmn + kTile;
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)  // K = 128 query rows, 16 per MMA
             mma_ts(tmem + TM_DV, tmem + TM_S + 64 * (kk >> 2) + 8 * (kk & 3), omn + kk * (2048 >> 4), idesc_g,
                    (j > 0 || kk > 0) ? 1u : 0u);
+          // S^T(g+1) overwrites P^T(g) after dV(g) has read it (same MMA stream)
+          if (j + 1 < n_tiles) issue_s(g + 1);
+          // dK(g) += dS^T(g) Q_g
+          mbar_wait(&bars->ds_ready[g & 1], (g >> 1) & 1, abort_flag);
+          tc_fence_after();
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)
             mma_ts(tmem + TM_DK, tmem + TM_DP + 64 * (kk >> 2) + 8 * (kk & 3), qmn + kk * (2048 >> 4), idesc_g,
@@ -279,6 +306,8 @@ __global__ void __launch_bounds__(384, 1)
           mma_commit(&bars->mma2_done[g & 1]);
           mma_commit(&bars->st_empty[st]);
           if (j + 1 == n_tiles) mma_commit(&bars->fix_empty);
+          // dP^T(g+1) overwrites dS^T(g) after dK(g) has read it
+          if (j + 1 < n_tiles) issue_dp(g + 1);
         }
         it += n_tiles;
       }
@@ -329,45 +358,70 @@ __global__ void __launch_bounds__(384, 1)
             mw[0] = mw[1] = mw[2] = mw[3] = 0u;
         }
         const uint32_t modes = partial ? chunk_modes(mw) : 0u;
+        // pass 1: P^T = exp2(S^T * scale*log2e - lse2), kept in fp32 for pass 2
         mbar_wait(&bars->s_full, g & 1, abort_flag);
         __syncwarp();
         tc_fence_after();
+        float pv[64];
 #pragma unroll
         for (int c = 0; c < 2; ++c) {
           const int gc = 2 * wg + c;  // 32-column chunk of the tile
           const uint32_t mode = (modes >> (2 * gc)) & 3u;
-          uint32_t pw[16], dw[16];
-          if (mode == 2u) {  // every lane of the warp masks this chunk: P^T = dS^T = 0
+          uint32_t pw[16];
+          if (mode == 2u) {  // every lane of the warp masks this chunk: P^T = 0
 #pragma unroll
-            for (int e = 0; e < 16; ++e) pw[e] = dw[e] = 0u;
+            for (int e = 0; e < 32; ++e) pv[32 * c + e] = 0.f;
+#pragma unroll
+            for (int e = 0; e < 16; ++e) pw[e] = 0u;
           } else {
-            uint32_t rs[32], rp[32];
+            uint32_t rs[32];
             tmem_ld32(tmem + lane_addr + TM_S + gc * 32, rs);
-            tmem_ld32(tmem + lane_addr + TM_DP + gc * 32, rp);
             tmem_wait_ld();
             const uint32_t bits = mode == 0u ? 0xffffffffu : mw[gc];
 #pragma unroll
-            for (int e = 0; e < 16; ++e) {
-              float pv[2], dv[2];
+            for (int e = 0; e < 32; ++e) {
+              const float x = fmaf(__uint_as_float(rs[e]), p.scale_log2, -vbuf[c * 32 + e]);
+              const float pe = ex2_approx(x);
+              pv[32 * c + e] = (mode == 0u || ((bits >> e) & 1u)) ? pe : 0.f;
+            }
 #pragma unroll
-              for (int z = 0; z < 2; ++z) {
-                const int ql = c * 32 + 2 * e + z;  // query index inside this warpgroup's 64
-                const float x = fmaf(__uint_as_float(rs[2 * e + z]), p.scale_log2, -vbuf[ql]);
-                pv[z] = ex2_approx(x);
-                if (mode != 0u) pv[z] = ((bits >> (2 * e + z)) & 1u) ? pv[z] : 0.f;
-                dv[z] = pv[z] * (__uint_as_float(rp[2 * e + z]) - vbuf[64 + ql]);
-              }
-              pw[e] = pack_bf16x2(pv[0], pv[1]);
-              dw[e] = pack_bf16x2(dv[0], dv[1]);
+            for (int e = 0; e < 16; ++e) pw[e] = pack_bf16x2(pv[32 * c + 2 * e], pv[32 * c + 2 * e + 1]);
+          }
+          // bf16 P^T goes to this warpgroup's own columns, over S^T it has already read
+          tmem_st16(tmem + lane_addr + TM_S + 64 * wg + c * 16, pw);
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(&bars->p_ready[g & 1]);
+        // pass 2: dS^T = P^T * (dP^T - Dr)
+        mbar_wait(&bars->dp_full, g & 1, abort_flag);
+        __syncwarp();
+        tc_fence_after();
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          const int gc = 2 * wg + c;
+          const uint32_t mode = (modes >> (2 * gc)) & 3u;
+          uint32_t dw[16];
+          if (mode == 2u) {
+#pragma unroll
+            for (int e = 0; e < 16; ++e) dw[e] = 0u;
+          } else {
+            uint32_t rp[32];
+            tmem_ld32(tmem + lane_addr + TM_DP + gc * 32, rp);
+            tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+              const int q0 = c * 32 + 2 * e;  // query index inside this warpgroup's 64
+              const float d0 = pv[q0] * (__uint_as_float(rp[2 * e]) - vbuf[64 + q0]);
+              const float d1 = pv[q0 + 1] * (__uint_as_float(rp[2 * e + 1]) - vbuf[64 + q0 + 1]);
+              dw[e] = pack_bf16x2(d0, d1);
             }
           }
-          // bf16 results go to this warpgroup's own columns, over data already read
-          tmem_st16(tmem + lane_addr + TM_S + 64 * wg + c * 16, pw);
           tmem_st16(tmem + lane_addr + TM_DP + 64 * wg + c * 16, dw);
         }
         tmem_wait_st();
         tc_fence_before();
-        mbar_arrive(&bars->ew_full[g & 1]);
+        mbar_arrive(&bars->ds_ready[g & 1]);
       }
       // epilogue: warpgroup 0 writes dK (scaled), warpgroup 1 writes dV
       const uint32_t g_last = it + n_tiles - 1;
