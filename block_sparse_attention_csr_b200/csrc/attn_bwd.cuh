@@ -651,11 +651,19 @@ __global__ void __launch_bounds__(384, 1)
           if (mode == 2u) {  // every lane of the warp masks this chunk: dS = 0
 #pragma unroll
             for (int e = 0; e < 16; ++e) dw[e] = 0u;
+            if (c == 1) {  // S and dP fully read: the next tile's S / dP may overwrite them
+              tc_fence_before();
+              mbar_arrive(&bars->s_free);
+            }
           } else {
             uint32_t rs[32], rp[32];
             tmem_ld32(tmem + lane_addr + TM_S + gc * 32, rs);
             tmem_ld32(tmem + lane_addr + TM_DP + gc * 32, rp);
             tmem_wait_ld();
+            if (c == 1) {  // S and dP fully read: the next tile's S / dP may overwrite them
+              tc_fence_before();
+              mbar_arrive(&bars->s_free);
+            }
             const uint32_t bits = mw[gc];
 #pragma unroll
             for (int e = 0; e < 16; ++e) {
@@ -673,7 +681,6 @@ __global__ void __launch_bounds__(384, 1)
         }
         tmem_wait_st();
         tc_fence_before();
-        mbar_arrive(&bars->s_free);
         mbar_arrive(&bars->ew_full[db]);
       }
       const uint32_t g_last = it + n_tiles - 1;
