@@ -24,7 +24,6 @@ from ._binding import (  # noqa: F401
     radial_mask_build_dense,
     radial_params_default,
     radial_selftest_bounded_wait,
-    radial_selftest_exp2,
 )
 
 TILE_FULL = 1

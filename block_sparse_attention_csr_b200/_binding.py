@@ -28,7 +28,7 @@ EXPORTED = (
     "radial_csr_copy_to_host", "radial_csr_free", "radial_attn_fwd",
     "radial_attn_bwd_workspace_size", "radial_attn_bwd", "radial_device_status",
     "radial_status_str", "radial_last_error", "radial_launch_count", "radial_selftest_bounded_wait",
-    "radial_selftest_exp2", "radial_attn_bwd_noalloc",
+    "radial_attn_bwd_noalloc",
 )
 
 
@@ -103,8 +103,6 @@ def load(path=None):
         L.radial_last_error.restype = ctypes.c_char_p
         L.radial_selftest_bounded_wait.argtypes = [ctypes.c_uint32, vp]
         L.radial_selftest_bounded_wait.restype = ctypes.c_int
-        L.radial_selftest_exp2.argtypes = [vp, vp, ctypes.c_int32, vp]
-        L.radial_selftest_exp2.restype = ctypes.c_int
         L.radial_launch_count.argtypes = []
         L.radial_launch_count.restype = i64
         _lib = L
@@ -286,13 +284,6 @@ def radial_device_status(stream=None):
 
 def radial_selftest_bounded_wait(limit_ms=20, stream=None):
     _check(load().radial_selftest_bounded_wait(int(limit_ms), _stream(stream)), "radial_selftest_bounded_wait")
-
-
-def radial_selftest_exp2(x, y=None, stream=None):
-    import torch
-    y = torch.empty_like(x) if y is None else y
-    _check(load().radial_selftest_exp2(_ptr(x), _ptr(y), int(x.numel()), _stream(stream)), "radial_selftest_exp2")
-    return y
 
 
 def radial_launch_count():

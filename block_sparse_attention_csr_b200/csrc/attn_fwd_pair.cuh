@@ -94,14 +94,6 @@ struct PairBars {
 };
 static_assert(sizeof(PairBars) <= 256, "barriers overlap the row exchange buffer");
 
-// Exponential pairs computed on the FMA pipe (exp2_poly_x2) instead of the
-// MUFU: bit e of the mask selects pair e of every 16-pair (32-key) chunk.
-// The MUFU issues 16 exponentials per clock and SM -- exactly what the tensor
-// core's 128x128x128 S and PV tiles need in the same time -- so a share on
-// the FMA pipe gives it headroom.
-constexpr uint32_t kPairPolyMask = 0u;
-__host__ __device__ constexpr bool use_poly_pair(int e) { return ((kPairPolyMask >> e) & 1u) != 0u; }
-
 template <int D>
 __global__ void __launch_bounds__(384, 1)
     radial_fwd_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -415,14 +407,9 @@ __global__ void __launch_bounds__(384, 1)
             for (int e = 0; e < 16; ++e) {
               const int k2 = 32 * c + 2 * e;
               const uint64_t xs = f2_fma(f2_pack(__uint_as_float(r[k2]), __uint_as_float(r[k2 + 1])), sl2, negm);
-              uint64_t pe;
-              if (use_poly_pair(e)) {
-                pe = exp2_poly_x2(xs);
-              } else {
-                float x0, x1;
-                f2_unpack(xs, x0, x1);
-                pe = f2_pack(ex2_approx(x0), ex2_approx(x1));
-              }
+              float x0, x1;
+              f2_unpack(xs, x0, x1);
+              const uint64_t pe = f2_pack(ex2_approx(x0), ex2_approx(x1));
               acc2[e & 1] = f2_add(acc2[e & 1], pe);
               float p0, p1;
               f2_unpack(pe, p0, p1);

@@ -44,17 +44,6 @@ __global__ void selftest_bounded_wait_kernel(uint64_t limit_ns, int* waited_out)
   if (threadIdx.x == 0) *waited_out = ok ? 0 : 1;
 }
 
-// Evaluates exp2_poly_x2 (the FMA-pipe exponential of the forward softmax)
-// on n inputs, for testing it against its error bound.
-__global__ void selftest_exp2_kernel(const float* __restrict__ x, float* __restrict__ y, int n) {
-  const int i = 2 * (blockIdx.x * blockDim.x + threadIdx.x);
-  if (i >= n) return;
-  const float a = x[i], b = (i + 1 < n) ? x[i + 1] : 0.f;
-  float r0, r1;
-  f2_unpack(exp2_poly_x2(f2_pack(a, b)), r0, r1);
-  y[i] = r0;
-  if (i + 1 < n) y[i + 1] = r1;
-}
 }  // namespace radial
 
 // ---------------------------------------------------------------------------
@@ -311,7 +300,13 @@ radial_status build_mask(int32_t f, int32_t s, int32_t B, int32_t sink, int32_t 
   radial_csr* c = new (std::nothrow) radial_csr();
   if (!c) return fail(RADIAL_ENOMEM, "host allocation failed");
   c->f = f; c->s = s; c->n = n; c->B = B; c->sink = sink; c->dense = dense;
-  cudaGetDevice(&c->device);
+  {
+    const cudaError_t e = cudaGetDevice(&c->device);
+    if (e != cudaSuccess) {
+      delete c;
+      return fail(RADIAL_ECUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
+    }
+  }
   if (!rule.is_default()) {
     std::vector<int32_t> H, C;
     if (!mask_rule_table(rule, f, s, H, C)) {
@@ -490,7 +485,7 @@ radial_status check_desc(const radial_csr* c, const radial_desc* d) {
   if (static_cast<int64_t>(d->batch) * d->heads * ((d->n_tokens + 127) / 128) > 0x7fffffffLL)
     return fail(RADIAL_EUNSUPPORTED, "too many work items");
   int dev = 0;
-  cudaGetDevice(&dev);
+  RADIAL_CUDA(cudaGetDevice(&dev));
   if (dev != c->device) return fail(RADIAL_EINVAL, "mask built on device %d, current device %d", c->device, dev);
   return RADIAL_OK;
 }
@@ -598,6 +593,18 @@ template <int D>
 radial_status launch_bwd(const radial_csr* c, const radial_desc* d, const void* dout, const void* q,
                          const void* k, const void* v, const void* o, const float* lse, void* dq, void* dk,
                          void* dv, float* dr, cudaStream_t st) {
+  // Everything that can fail on the host (tensor maps, kernel attributes)
+  // happens before the first launch: a call that returns an error has
+  // launched nothing and left the workspace untouched.
+  CUtensorMap mq, mk, mv, mdo;
+  radial_status rs;
+  if ((rs = make_bhnd_map(&mq, q, *d)) != RADIAL_OK) return rs;
+  if ((rs = make_bhnd_map(&mk, k, *d)) != RADIAL_OK) return rs;
+  if ((rs = make_bhnd_map(&mv, v, *d)) != RADIAL_OK) return rs;
+  if ((rs = make_bhnd_map(&mdo, dout, *d)) != RADIAL_OK) return rs;
+  const int smem = BwdCfg<D>::SMEM_BYTES;
+  RADIAL_CUDA(cudaFuncSetAttribute(radial_bwd_dkdv_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
+  RADIAL_CUDA(cudaFuncSetAttribute(radial_bwd_dq_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
   const int64_t rows = static_cast<int64_t>(d->batch) * d->heads * d->n_tokens;
   {
     const int threads = 256;
@@ -607,12 +614,6 @@ radial_status launch_bwd(const radial_csr* c, const radial_desc* d, const void* 
         d->n_tokens, d->stride_b, d->stride_h, d->stride_n, rows, dr);
     RADIAL_LAUNCHED();
   }
-  CUtensorMap mq, mk, mv, mdo;
-  radial_status rs;
-  if ((rs = make_bhnd_map(&mq, q, *d)) != RADIAL_OK) return rs;
-  if ((rs = make_bhnd_map(&mk, k, *d)) != RADIAL_OK) return rs;
-  if ((rs = make_bhnd_map(&mv, v, *d)) != RADIAL_OK) return rs;
-  if ((rs = make_bhnd_map(&mdo, dout, *d)) != RADIAL_OK) return rs;
   BwdParams p;
   p.row_ptr = c->plan.row_ptr;
   p.col_idx = c->plan.col_idx;
@@ -641,9 +642,6 @@ radial_status launch_bwd(const radial_csr* c, const radial_desc* d, const void* 
   p.dv = reinterpret_cast<__nv_bfloat16*>(dv);
   p.scale = softmax_scale(d);
   p.scale_log2 = p.scale * 1.4426950408889634f;
-  const int smem = BwdCfg<D>::SMEM_BYTES;
-  RADIAL_CUDA(cudaFuncSetAttribute(radial_bwd_dkdv_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
-  RADIAL_CUDA(cudaFuncSetAttribute(radial_bwd_dq_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
   const int grid = p.items < sm_count() ? p.items : sm_count();
   radial_bwd_dkdv_kernel<D><<<grid, 384, smem, st>>>(mq, mk, mv, mdo, p);
   RADIAL_LAUNCHED();
@@ -786,15 +784,6 @@ radial_status radial_selftest_bounded_wait(uint32_t limit_ms, void* stream) {
   cudaFree(flag);
   if (e != cudaSuccess) return fail(RADIAL_ECUDA, "self-test: %s", cudaGetErrorString(e));
   if (h != 1) return fail(RADIAL_ECUDA, "self-test: the wait did not time out");
-  return RADIAL_OK;
-}
-
-radial_status radial_selftest_exp2(const float* x, float* y, int32_t n, void* stream) {
-  if (!x || !y || n < 1) return fail(RADIAL_EINVAL, "bad arguments");
-  const int threads = 256;
-  const int blocks = ((n + 1) / 2 + threads - 1) / threads;
-  selftest_exp2_kernel<<<blocks, threads, 0, as_stream(stream)>>>(x, y, n);
-  RADIAL_LAUNCHED();
   return RADIAL_OK;
 }
 

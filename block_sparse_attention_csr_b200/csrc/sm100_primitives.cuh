@@ -299,38 +299,6 @@ __device__ __forceinline__ float max3f(float a, float b, float c) {
   return d;
 }
 
-// 2^x for two lanes on the FMA / integer pipes (no MUFU): x = j + f with
-// j = round(x) (obtained by adding 1.5 * 2^23, which leaves j in the low
-// mantissa bits) and f in [-1/2, 1/2]; 2^f from a cubic whose relative error
-// is below 7.5e-5 (coefficients from gen_exp2_poly.py: Lawson-weighted least
-// squares, i.e. near-minimax in relative error); 2^j is added to the
-// exponent field.  Inputs are clamped at -125 so the result stays a normal
-// float (about 2.4e-38 for any smaller input, e.g. -inf from the mask).
-__device__ __forceinline__ uint64_t exp2_poly_x2(uint64_t x) {
-  float x0, x1;
-  f2_unpack(x, x0, x1);
-  x0 = fmaxf(x0, -125.0f);
-  x1 = fmaxf(x1, -125.0f);
-  const uint64_t xx = f2_pack(x0, x1);
-  const uint64_t kShift = f2_pack(12582912.0f, 12582912.0f);   // 1.5 * 2^23
-  const uint64_t kNegShift = f2_pack(-12582912.0f, -12582912.0f);
-  const uint64_t kNegOne = f2_pack(-1.0f, -1.0f);
-  const uint64_t t = f2_add(xx, kShift);
-  const uint64_t r = f2_add(t, kNegShift);        // round(x) as a float
-  const uint64_t f = f2_fma(r, kNegOne, xx);      // x - round(x)
-  uint64_t q = f2_fma(f2_pack(0.055171526968479156f, 0.055171526968479156f), f,
-                      f2_pack(0.24261116981506348f, 0.24261116981506348f));
-  q = f2_fma(q, f, f2_pack(0.6932610273361206f, 0.6932610273361206f));
-  q = f2_fma(q, f, f2_pack(0.9999280571937561f, 0.9999280571937561f));
-  float t0, t1, q0, q1;
-  f2_unpack(t, t0, t1);
-  f2_unpack(q, q0, q1);
-  const int j0 = __float_as_int(t0) - 0x4B400000;
-  const int j1 = __float_as_int(t1) - 0x4B400000;
-  return f2_pack(__int_as_float(__float_as_int(q0) + (j0 << 23)),
-                 __int_as_float(__float_as_int(q1) + (j1 << 23)));
-}
-
 // Named barrier over the first `nthreads` threads that reach barrier `id`
 // (ids 1..15; 0 is __syncthreads).
 __device__ __forceinline__ void named_bar_sync(int id, int nthreads) {

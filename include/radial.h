@@ -190,7 +190,10 @@ radial_status radial_attn_bwd(const radial_csr* csr, const radial_desc* desc, co
  * nothing.  The call allocates nothing: no cudaMalloc, no cudaFree, no
  * allocating library routine.  The first call on a device looks up the
  * array's device address (cudaGetSymbolAddress, once per device, with that
- * device current); make that first call before any stream capture.  Every
+ * device current) and keeps it for the life of the process; make that first
+ * call before any stream capture, and do not use this call on a device after
+ * cudaDeviceReset (the reset unloads the module, and the kept address would
+ * then name memory the library no longer owns).  Every
  * call shares the one array per device, which keeps the last call's contents
  * (each call overwrites every row it reads before reading it), so calls that
  * overlap on the GPU, on different streams or threads, race and must be
@@ -212,12 +215,6 @@ radial_status radial_device_status(void* stream);
  * the context stays usable.  Synchronous.  RADIAL_OK if the wait timed out
  * as designed. */
 radial_status radial_selftest_bounded_wait(uint32_t limit_ms, void* stream);
-
-/* Self-test of the polynomial base-2 exponential that the forward softmax
- * can run on the FMA pipe for part of its elements (a compile-time switch,
- * off by default: measured no faster than the MUFU alone): y[i] = 2^x[i] for
- * n device floats (inputs below -125 give about 2^-125).  Asynchronous. */
-radial_status radial_selftest_exp2(const float* x, float* y, int32_t n, void* stream);
 
 /* Static text for a status code. */
 const char* radial_status_str(radial_status s);
