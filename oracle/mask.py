@@ -28,8 +28,12 @@ Width below one ([review] Fig.5 caption and Eq.4 case (ii); [rebuttal]
 ``w(d) = 0`` (``h(d) < 0``) only the main diagonal ``k == l`` is kept, and only
 in every ``c(d)``-th frame pair, ``c(d) = ceil(2**r(d) / s)``, so the amortised
 density keeps halving per band.  The exact subsampling rule is not printed;
-``d mod c(d) == 0`` is the plainest reading.  PARITY UNPINNED beyond the
-invariants tested (it never triggers at the benchmark shapes).
+``d mod c(d) == 0`` is the plainest reading.  What the pages do state -- the
+amortised density keeps halving per band and only the main diagonal is kept
+-- is pinned by brute-force band counts (tests/test_oracle_mask.py); which
+frame pairs of a band carry the kept diagonal (the phase of ``d mod c``) is
+the one choice the pages leave open.  The branch never triggers at the
+benchmark shapes.
 
 Attention sink ([review] §4.2 and App. A.1 Eq.8): every query also attends
 to every token of frame 0 (key frame ``j == 0``).  Query rows of frame 0 are

@@ -242,12 +242,58 @@ def test_sampling_branch_reached_on_tiny_grid():
     assert (blk == np.eye(s, dtype=bool)).all()
     # frame distance 9: c = 2 -> not on the period -> nothing
     assert not m[0:s, 9 * s:10 * s].any()
-    # amortised density still halves per band: band r has 2^r distances,
-    # every c-th kept with s pairs -> about s * 2^r / c = s^2 pairs per band
-    for r in range(3, 6):
-        ds = range(2 ** r, 2 ** (r + 1))
-        kept = sum(int(m[0:s, d * s:(d + 1) * s].sum()) for d in ds)
-        assert kept == sum(s for d in ds if d % int(M.sample_period(d, s)) == 0)
+
+
+def _band_sums(f, s):
+    """Kept pairs per temporal band, counted on the brute-force token mask
+    (sink off): B(r) = sum over the band's distances d in [2^r, 2^(r+1)) of
+    the allowed (k, l) pairs between frame 0 and frame d."""
+    m = M.token_mask(f, s, sink=False)
+    per_d = np.array([int(m[0:s, d * s:(d + 1) * s].sum()) for d in range(f)])
+    sums = {}
+    r = 1
+    while 2 ** (r + 1) <= f:
+        sums[r] = int(per_d[2 ** r:2 ** (r + 1)].sum())
+        r += 1
+    return per_d, sums
+
+
+@pytest.mark.parametrize("f,s", [(256, 4), (256, 3), (512, 5), (128, 2)])
+def test_sampled_diagonal_keeps_the_amortised_density_decay(f, s):
+    """[review] Fig.5 caption and [rebuttal] (diagonal frequency reduction):
+    once a band's diagonal width falls below one token, frame pairs are
+    subsampled so that the AMORTISED density keeps decaying as before, i.e.
+    it keeps halving from one temporal band to the next, and what is kept is
+    the main diagonal only.  Counted by brute force, independent of the rule
+    that produces it: the band's density rho(r) = B(r) / (2^r s^2) must halve
+    per band (ratio within [1/3, 1] once ceil rounding is allowed for), and
+    the kept pairs per band, B(r) = rho(r) 2^r s^2, stay between 3/4 and 2
+    times those of the last band whose width is still one token (that band
+    holds 2^r s pairs with s/2 < 2^r <= s; a halving density keeps B(r) near
+    s^2 from then on).  A rule that keeps the
+    diagonal in every pair (density stops falling), in no pair, or subsampled
+    by 2^r instead of 2^r / s (density falls s times too fast) fails here."""
+    per_d, sums = _band_sums(f, s)
+    widths = {r: s // 2 ** r for r in sums}
+    sampled = [r for r in sums if widths[r] == 0]
+    last_w1 = max(r for r in sums if widths[r] == 1)
+    assert len(sampled) >= 3, "grid too small to reach several sampled bands"
+    rho = {r: sums[r] / (2 ** r * s * s) for r in sums}
+    for r in [last_w1] + sampled:
+        if r - 1 in rho and widths[r - 1] <= 1:
+            ratio = rho[r] / rho[r - 1]
+            assert 1.0 / 3.0 <= ratio <= 1.0, (r, ratio)
+    for r in sampled:
+        assert 0.75 * sums[last_w1] <= sums[r] <= 2 * sums[last_w1], (r, sums[r], sums[last_w1])
+    # the pages describe diagonal samples: in a sampled band a kept frame pair
+    # holds the main diagonal k == l and nothing else
+    m = M.token_mask(f, s, sink=False)
+    for r in sampled:
+        for d in range(2 ** r, 2 ** (r + 1)):
+            blk = m[0:s, d * s:(d + 1) * s]
+            assert (not blk.any()) or (blk == np.eye(s, dtype=bool)).all(), d
+    # and the total still grows like n log n: band sums do not grow with r
+    assert max(sums[r] for r in sampled) <= 2 * s * s
 
 
 @pytest.mark.parametrize("f,s,sink", [(8, 16, True), (64, 4, False), (64, 4, True), (9, 7, True), (1, 5, False)])
