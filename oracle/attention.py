@@ -8,7 +8,11 @@ attention of [review] §3 Eq.2, ``O = softmax(Q K^T * scale + M) V`` with
 ``M`` = 0 on allowed pairs and -inf elsewhere; its block-sparse execution
 ([review] §4.2, 128x128 blocks) only skips tiles where ``M`` is -inf
 everywhere.  So this module is that definition written out, with no blocking,
-fusion or reordering.  The pages fix neither the scale nor the saved
+fusion or reordering.  The whole-head functions at the end evaluate each
+chunk of rows against a superset of its allowed keys (mask.key_superset):
+the keys they leave out are masked for every row of the chunk and would add
+exp(-inf) = 0 to each sum, so the result is the same definition; the tests
+pin them to the dense evaluation.  The pages fix neither the scale nor the saved
 statistics; the readings taken: ``scale = 1/sqrt(d)`` (the Eq.1 convention),
 ``LSE`` = natural-log log-sum-exp of the masked, scaled logits per row.
 
@@ -175,3 +179,116 @@ def sample_rows(n, count, s, B, seed):
     extra = rng.choice(n, size=min(n, count * 2), replace=False)
     extra = np.setdiff1d(extra, fixed)[: count - fixed.size]
     return np.sort(np.concatenate([fixed, extra]))
+
+
+# ---------------------------------------------------------------------------
+# Whole-head statistics and key-column gradients (dK, dV at large shapes)
+# ---------------------------------------------------------------------------
+
+def _chunks_in_frames(n, s, chunk):
+    """Consecutive row ranges [a0, a1) of at most `chunk` rows, none crossing
+    a frame boundary."""
+    out = []
+    for f0 in range(0, n, s):
+        f1 = min(n, f0 + s)
+        for a0 in range(f0, f1, chunk):
+            out.append((a0, min(f1, a0 + chunk)))
+    return out
+
+
+def head_row_stats(q, k, v, do, f, s, sink=True, scale=None, chunk=128, threads=None, spec=None):
+    """LSE and Dr = rowsum(dO * O) of EVERY query row of one (batch, head).
+
+    Each chunk of consecutive rows of one frame is Eq.2 evaluated against
+    the key superset of mask.key_superset(): the keys left out are masked
+    for every row of the chunk, so they contribute exp(-inf) = 0 to every
+    sum and leaving them out changes neither LSE nor O.  q, k, v, do: (n, d)
+    arrays (any float dtype; the arithmetic is fp64).  Chunks run on a thread
+    pool (NumPy releases the interpreter lock inside its kernels)."""
+    import os
+    from concurrent.futures import ThreadPoolExecutor
+
+    n, dh = q.shape
+    scale = 1.0 / np.sqrt(dh) if scale is None else scale
+    q, k, v, do = (_as64(x) for x in (q, k, v, do))
+    lse = np.empty(n)
+    dr = np.empty(n)
+
+    def work(rng):
+        a0, a1 = rng
+        keys = _mask.key_superset(a0, a1, f, s, sink, spec)
+        rows = np.arange(a0, a1, dtype=np.int64)
+        S = (q[a0:a1] @ k[keys].T) * scale
+        S = np.where(_mask.pair_mask(rows, keys, f, s, sink, spec), S, -np.inf)
+        m = S.max(axis=1, keepdims=True)
+        P = np.exp(S - m)
+        l = P.sum(axis=1, keepdims=True)
+        o = (P @ v[keys]) / l
+        lse[a0:a1] = m[:, 0] + np.log(l[:, 0])
+        dr[a0:a1] = (do[a0:a1] * o).sum(axis=1)
+
+    ranges = _chunks_in_frames(n, s, chunk)
+    threads = threads or max(1, len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else 1)
+    try:
+        from threadpoolctl import threadpool_limits
+        limiter = threadpool_limits(1)
+    except Exception:  # pragma: no cover - threadpoolctl is optional
+        limiter = None
+    try:
+        with ThreadPoolExecutor(threads) as ex:
+            list(ex.map(work, ranges))
+    finally:
+        if limiter is not None:
+            limiter.restore_original_limits()
+    return lse, dr
+
+
+def dkdv_cols(q, k, v, do, lse, dr, cols, f, s, sink=True, scale=None, chunk=8192, threads=None, spec=None):
+    """dK and dV of the given key columns of one (batch, head).
+
+    Column b of the gradients is a sum over every query a:
+        P[a, b] = exp(S[a, b] - LSE[a])  (0 where (a, b) is masked)
+        dV[b]   = sum_a P[a, b] dO[a]
+        dS[a, b] = P[a, b] (dO[a] . V[b] - Dr[a])
+        dK[b]   = scale * sum_a dS[a, b] Q[a]
+    with the row statistics LSE and Dr of every query (head_row_stats or the
+    dense forward).  Queries are taken in chunks; the result is a plain sum
+    over them (chunks on a thread pool, partial sums added in query order).
+    Returns (dK_cols, dV_cols), each (len(cols), d)."""
+    import os
+    from concurrent.futures import ThreadPoolExecutor
+
+    n, dh = q.shape
+    scale = 1.0 / np.sqrt(dh) if scale is None else scale
+    cols = np.asarray(cols, dtype=np.int64)
+    kc, vc = _as64(k[cols]), _as64(v[cols])
+
+    def part(a0):
+        a1 = min(n, a0 + chunk)
+        rows = np.arange(a0, a1, dtype=np.int64)
+        qa, doa = _as64(q[a0:a1]), _as64(do[a0:a1])
+        S = (qa @ kc.T) * scale
+        with np.errstate(invalid="ignore", over="ignore"):
+            P = np.where(_mask.pair_mask(rows, cols, f, s, sink, spec),
+                         np.exp(S - _as64(lse[a0:a1])[:, None]), 0.0)
+        dS = P * (doa @ vc.T - _as64(dr[a0:a1])[:, None])
+        return dS.T @ qa, P.T @ doa
+
+    threads = threads or max(1, len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else 1)
+    try:
+        from threadpoolctl import threadpool_limits
+        limiter = threadpool_limits(1)
+    except Exception:  # pragma: no cover - threadpoolctl is optional
+        limiter = None
+    try:
+        with ThreadPoolExecutor(threads) as ex:
+            parts = list(ex.map(part, range(0, n, chunk)))   # in query order
+    finally:
+        if limiter is not None:
+            limiter.restore_original_limits()
+    dK = np.zeros((cols.size, dh))
+    dV = np.zeros((cols.size, dh))
+    for pk, pv in parts:
+        dK += pk
+        dV += pv
+    return scale * dK, dV

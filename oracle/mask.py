@@ -206,6 +206,17 @@ def _mask_from_table(qi, qk, kj, kl, f, s, sink, spec=None):
     H, Cp = distance_table(f, s) if spec is None else spec_distance_table(f, s, spec)
     H = H.astype(np.int32)
     Cp = Cp.astype(np.int32)
+    if qi.size and (qi == qi[0]).all():
+        # every query in one frame: d, h(d), c(d) depend on the key alone
+        d1 = np.abs(qi[0] - kj)
+        h1 = H[d1]
+        out = np.abs(qk[:, None] - kl[None, :]) <= h1[None, :]      # h < 0 never passes
+        samp = (h1 < 0) & (d1 % Cp[d1] == 0)
+        if samp.any():
+            out[:, samp] |= qk[:, None] == kl[samp][None, :]
+        if sink:
+            out[:, kj == 0] = True
+        return out
     d = np.abs(qi[:, None] - kj[None, :])
     h = H[d]
     out = np.abs(qk[:, None] - kl[None, :]) <= h          # h < 0 never passes
@@ -231,6 +242,44 @@ def col_mask(cols, f, s, sink=True, spec=None):
     cols = np.asarray(cols, dtype=np.int32)
     a = np.arange(n, dtype=np.int32)
     return _mask_from_table(a // s, a % s, cols // s, cols % s, f, s, sink, spec)
+
+
+def pair_mask(rows, cols, f, s, sink=True, spec=None):
+    """Boolean mask of the given query rows against the given key columns."""
+    rows = np.asarray(rows, dtype=np.int32)
+    cols = np.asarray(cols, dtype=np.int32)
+    return _mask_from_table(rows // s, rows % s, cols // s, cols % s, f, s, sink, spec)
+
+
+def key_superset(a0, a1, f, s, sink=True, spec=None):
+    """Key indices (sorted, int64) that include every key any query row in
+    [a0, a1) may attend to.  The rows must lie in one frame i.
+
+    Per key frame j the allowed keys of row (i, k) are, by the rule of
+    allowed(): all of frame 0 (sink), the window |k - l| <= h(d), the single
+    position l = k (sampled diagonal, on its period), or nothing.  Over
+    k in [k0, k1] their union lies inside [k0 - h, k1 + h] (or [k0, k1]),
+    clipped to the frame; those ranges are returned.  Used to skip keys whose
+    logits are masked for every row of a chunk -- they would only add
+    exp(-inf) = 0 to each sum -- when the oracle evaluates whole heads."""
+    i = a0 // s
+    assert 0 <= a0 < a1 <= (i + 1) * s, "rows must lie in one frame"
+    k0, k1 = a0 - i * s, a1 - 1 - i * s
+    H, Cp = distance_table(f, s) if spec is None else spec_distance_table(f, s, spec)
+    parts = []
+    for j in range(f):
+        d = abs(i - j)
+        h, c = int(H[d]), int(Cp[d])
+        if sink and j == 0:
+            lo, hi = 0, s - 1
+        elif h >= 0:
+            lo, hi = max(0, k0 - h), min(s - 1, k1 + h)
+        elif d % c == 0:
+            lo, hi = k0, k1
+        else:
+            continue
+        parts.append(np.arange(j * s + lo, j * s + hi + 1, dtype=np.int64))
+    return np.concatenate(parts) if parts else np.zeros(0, dtype=np.int64)
 
 
 # ---------------------------------------------------------------------------

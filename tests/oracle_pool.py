@@ -42,6 +42,17 @@ def _dq_rows(args):
     return A.dq_rows(q, k, v, do, rows, f, s, sink, scale)
 
 
+def _bwd_head(args):
+    """Forward and backward of one whole (batch, head) by the dense reference."""
+    from oracle import attention as A
+    from oracle import mask as M
+    q, k, v, do, f, s, sink = args
+    scale = 1.0 / np.sqrt(q.shape[1])
+    allowed = M.token_mask(f, s, sink)
+    o, lse = A.forward(q, k, v, allowed, scale)
+    return A.backward(q, k, v, o, do, lse, allowed, scale)
+
+
 def cores():
     try:
         return len(os.sched_getaffinity(0))
@@ -50,7 +61,7 @@ def cores():
 
 
 def run(fn_name, tasks, workers=None):
-    fn = {"fwd_rows": _fwd_rows, "dq_rows": _dq_rows}[fn_name]
+    fn = {"fwd_rows": _fwd_rows, "dq_rows": _dq_rows, "bwd_head": _bwd_head}[fn_name]
     if not tasks:
         return []
     c = cores()

@@ -90,7 +90,23 @@ def test_backward_is_deterministic():
         assert torch.equal(x, y)
 
 
-def _large_check(name, rows_per_head):
+def test_many_work_items_all_gradients():
+    """8 heads x 71 key (and query) tiles = 568 work items per backward kernel,
+    several per persistent CTA on 148 SMs: every element of dQ, dK and dV
+    against the dense reference, head by head."""
+    wl = I.small_workload("bmany", 1, 8, 128, 9, 1000, 128, 42)
+    q, k, v, do = I.draw(wl, device=DEV, backward=True)
+    csr = rb.radial_mask_build(9, 1000, 128, sink=1)
+    _, _, dq, dk, dv = _gpu_fwd_bwd(q, k, v, do, csr)
+    x = [t[0].double().cpu().numpy() for t in (q, k, v, do)]
+    ref = oracle_pool.run("bwd_head", [(x[0][h], x[1][h], x[2][h], x[3][h], 9, 1000, True) for h in range(8)])
+    for h, (rq, rk, rv) in enumerate(ref):
+        for name, g, r in zip(("dQ", "dK", "dV"), (dq, dk, dv), (rq, rk, rv)):
+            err = np.abs(g[0, h].double().cpu().numpy() - r).max()
+            assert err <= G_MAX, f"head {h}: {name} max-abs {err:.3e}"
+
+
+def _large_check(name, rows_per_head, dkdv_heads, cols_per_head):
     wl = I.WORKLOADS[name]
     q, k, v, do = I.draw(wl, device=DEV, backward=True)
     csr = rb.radial_mask_build(wl.frames, wl.tokens_per_frame, wl.block, sink=1)
@@ -104,9 +120,23 @@ def _large_check(name, rows_per_head):
     # bf16 storage of each term (2^-9 relative) plus the bf16 O inside rowsum(dO o O)
     assert (dk64.abs() <= 2.0 ** -7 * dk_scale + 1e-3).all(), "sum_k dK != 0"
     assert ((dv64 - do64).abs() <= 2.0 ** -7 * dv_scale + 1e-3).all(), "sum_k dV != sum_q dO"
-    # sampled dQ rows against the reference
-    tasks, got = [], []
     scale = 1.0 / np.sqrt(wl.head_dim)
+    # dK / dV on sampled key columns of seeded heads: every query's LSE and
+    # rowsum(dO o O) of those heads recomputed in fp64 by the reference
+    rng = np.random.default_rng(3000 + wl.seed)
+    for h in sorted(rng.choice(wl.heads, size=dkdv_heads, replace=False).tolist()):
+        cols = A.sample_rows(wl.n, cols_per_head, wl.tokens_per_frame, wl.block, seed=4000 + h)
+        hq, hk, hv, hdo = (t[0, h].double().cpu().numpy() for t in (q, k, v, do))
+        lse_ref, dr_ref = A.head_row_stats(hq, hk, hv, hdo, wl.frames, wl.tokens_per_frame, True, scale)
+        dk_ref, dv_ref = A.dkdv_cols(hq, hk, hv, hdo, lse_ref, dr_ref, cols, wl.frames, wl.tokens_per_frame,
+                                     True, scale)
+        cidx = torch.as_tensor(cols, device=DEV)
+        for nm, g, r in (("dK", dk, dk_ref), ("dV", dv, dv_ref)):
+            err = np.abs(g[0, h, cidx].double().cpu().numpy() - r).max()
+            assert err <= G_MAX, f"{name} head {h}: {nm} max-abs {err:.3e} on {len(cols)} key columns"
+        del hq, hk, hv, hdo
+    # sampled dQ rows against the reference, every head
+    tasks, got = [], []
     for h in range(wl.heads):
         rows = A.sample_rows(wl.n, rows_per_head, wl.tokens_per_frame, wl.block, seed=2000 + h)
         ridx = torch.as_tensor(rows, device=DEV)
@@ -120,9 +150,11 @@ def _large_check(name, rows_per_head):
 
 
 def test_hunyuan720p_backward_sampled():
-    _large_check("hunyuan720p", int(os.environ.get("RADIAL_BWD_ROWS", "512")))
+    _large_check("hunyuan720p", int(os.environ.get("RADIAL_BWD_ROWS", "4096")), 2,
+                 int(os.environ.get("RADIAL_BWD_COLS", "4096")))
 
 
 @pytest.mark.slow
 def test_hunyuan720p_4x_backward_sampled():
-    _large_check("hunyuan720p_4x", int(os.environ.get("RADIAL_4X_BWD_ROWS", "1024")))
+    _large_check("hunyuan720p_4x", int(os.environ.get("RADIAL_4X_BWD_ROWS", "4096")),
+                 int(os.environ.get("RADIAL_4X_DKDV_HEADS", "2")), int(os.environ.get("RADIAL_4X_BWD_COLS", "4096")))

@@ -146,6 +146,28 @@ def test_hunyuan720p_4x_sampled_rows():
     _sampled_check("hunyuan720p_4x", int(os.environ.get("RADIAL_4X_ROWS", "4096")))
 
 
+@pytest.mark.parametrize("frames", [8, 16, 66])
+def test_sweep_sampled_rows(frames):
+    """The scaling sweep's other frame counts (33 and 132 are the HunyuanVideo
+    shapes above): 4096 sampled rows of every head."""
+    _sampled_check(f"sweep_f{frames}", int(os.environ.get("RADIAL_SWEEP_ROWS", "4096")))
+
+
+def test_many_work_items_all_rows():
+    """8 heads x 36 query-tile pairs = 288 work items, about two per
+    persistent CTA: every row of O and LSE against the reference."""
+    wl = I.small_workload("fmany", 1, 8, 128, 9, 1000, 128, 24)
+    q, k, v = I.draw(wl, device=DEV, backward=False)
+    o, lse = _run_gpu(q, k, v, 9, 1000, 128, 1)
+    rows = np.arange(wl.n)
+    scale = 1.0 / np.sqrt(wl.head_dim)
+    tasks = [(q[0, h].double().cpu().numpy(), k[0, h].float().cpu().numpy(), v[0, h].float().cpu().numpy(),
+              rows, 9, 1000, True, scale) for h in range(8)]
+    res = oracle_pool.run("fwd_rows", tasks)
+    _check(o[0].float().cpu().numpy().reshape(-1, 128), lse[0].cpu().numpy().reshape(-1),
+           np.concatenate([a for a, _ in res]), np.concatenate([b for _, b in res]), "many items")
+
+
 def test_one_tile_kernel_all_rows():
     """The alternate forward (one query tile per CTA, double-buffered S),
     selected per process by RADIAL_FWD_KERNEL=single: the all-row parity
