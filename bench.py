@@ -8,9 +8,11 @@ static mask is built once per shape (it depends on positions only) and its
 build time is reported beside the step.  With --workload hunyuan720p_4x a
 step is the 4x-length LoRA fine-tuning pass: forward plus backward.
 
-Prints one JSON line (rank 0).  Multi-GPU (torchrun): every rank runs the
-same workload on its own GPU (independent problems, no collective on the data
-path; weak scaling); the step time is the max over ranks.
+Prints one JSON line (rank 0).  Multi-GPU (torchrun): by default the one
+problem is split across the ranks by heads (rank r runs heads
+[r*H/N, (r+1)*H/N) on views of the same tensors; no collective on the data
+path; strong scaling); --shard replica runs one full replica per rank instead
+(weak scaling).  The step time is the max over ranks.
 
 --impl reference times the CPU reference (oracle/) on the host cores instead.
 """
@@ -53,11 +55,12 @@ def _cores():
 # workload accounting (host-side integers only)
 # ---------------------------------------------------------------------------
 
-def tile_flops(wl, nnz, backward=False):
+def tile_flops(wl, nnz, backward=False, heads=None):
     """Algorithmic flops on active tiles: 4*B^2*d per tile forward (QK^T and PV),
     10*B^2*d backward (five tile GEMMs), times batch*heads."""
     per = 4 if not backward else 10
-    return per * wl.block * wl.block * wl.head_dim * nnz * wl.batch * wl.heads
+    heads = wl.heads if heads is None else heads
+    return per * wl.block * wl.block * wl.head_dim * nnz * wl.batch * heads
 
 
 def whole_job_tflops(flops_per_rank, world, ms_max):
@@ -65,6 +68,12 @@ def whole_job_tflops(flops_per_rank, world, ms_max):
     (independent problems), so the job does world * flops_per_rank in the
     slowest rank's time."""
     return world * flops_per_rank / (ms_max * 1e-3) / 1e12
+
+
+def job_tflops(flops_total, ms_max):
+    """Whole-job throughput of one problem split across ranks: the problem's
+    flops in the slowest rank's time."""
+    return flops_total / (ms_max * 1e-3) / 1e12
 
 
 def max_over_ranks(ms, world, device=None):
@@ -198,7 +207,8 @@ def run_ours(args, rank, world, local_rank):
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
     wl = I.WORKLOADS[args.workload]
-    backward = wl.backward
+    step_kind = args.step or ("fwdbwd" if wl.backward else "fwd")
+    backward = step_kind != "fwd"
     peak, peak_sus, hbm, peak_src = _peaks()
     stream = torch.cuda.current_stream(dev)
 
@@ -213,14 +223,31 @@ def run_ours(args, rank, world, local_rank):
 
     q, k, v, *rest = I.draw(wl, device=dev, backward=True)
     do = rest[0]
-    o = torch.empty_like(q)
-    lse = torch.empty(q.shape[:3], dtype=torch.float32, device=dev)
+    heads_mode = args.shard == "heads"
+    h0, h1 = (0, wl.heads)
+    local = (lambda t: t)
+    if heads_mode and world > 1:
+        # this rank's heads of the one problem: views of the full tensors
+        from block_sparse_attention_csr_b200 import sharding
+        h0, h1 = sharding.head_range(wl.heads, world, rank)
+        local = (lambda t: sharding.shard(t, world, rank))
+    local_heads = h1 - h0
+    o = local(torch.empty_like(q))
     if backward:
-        dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
-        ws = torch.empty(rb.radial_attn_bwd_workspace_size(q), dtype=torch.uint8, device=dev)
+        dq, dk, dv = (local(torch.empty_like(t)) for t in (q, k, v))
+    q, k, v, do = (local(t) for t in (q, k, v, do))
+    lse = torch.empty(q.shape[:3], dtype=torch.float32, device=dev)   # [B, local heads, N], contiguous
+    if backward:
+        ws = torch.empty(max(256, rb.radial_attn_bwd_workspace_size(q)), dtype=torch.uint8, device=dev)
+
+    if step_kind == "bwd" and local_heads > 0:
+        rb.radial_attn_fwd(csr, q, k, v, o=o, lse=lse, stream=stream)   # O and LSE the backward reads
 
     def step():
-        rb.radial_attn_fwd(csr, q, k, v, o=o, lse=lse, stream=stream)
+        if local_heads == 0:  # more ranks than heads: this rank has nothing to run
+            return
+        if step_kind != "bwd":
+            rb.radial_attn_fwd(csr, q, k, v, o=o, lse=lse, stream=stream)
         if backward:
             rb.radial_attn_bwd(csr, do, q, k, v, o, lse, dq, dk, dv, ws, stream=stream)
 
@@ -259,8 +286,14 @@ def run_ours(args, rank, world, local_rank):
     ms = float(np.mean(step_ms))
     ms_max = max_over_ranks(ms, world, dev)
 
-    flops_step = tile_flops(wl, nnz) + (tile_flops(wl, nnz, True) if backward else 0)
-    value = whole_job_tflops(flops_step, world, ms_max)
+    with_fwd = step_kind != "bwd"
+    flops_step = (tile_flops(wl, nnz, heads=local_heads) if with_fwd else 0) + \
+        (tile_flops(wl, nnz, True, local_heads) if backward else 0)
+    if heads_mode:
+        value = job_tflops((tile_flops(wl, nnz) if with_fwd else 0) + (tile_flops(wl, nnz, True) if backward else 0),
+                           ms_max)
+    else:
+        value = whole_job_tflops(flops_step, world, ms_max)
 
     # forward kernel alone (dominant kernel of the default step) for the roofline
     fwd_ms = ms
@@ -272,10 +305,10 @@ def run_ours(args, rank, world, local_rank):
             b.record(stream)
         torch.cuda.synchronize(dev)
         fwd_ms = float(np.mean([a.elapsed_time(b) for a, b in e]))
-    fwd_tf = tile_flops(wl, nnz) / (fwd_ms * 1e-3) / 1e12
+    fwd_tf = tile_flops(wl, nnz, heads=local_heads) / (fwd_ms * 1e-3) / 1e12
 
     extra = {}
-    if rank == 0 and not args.quick:
+    if rank == 0 and not args.quick and world == 1:
         # dense comparator: same kernels, all-ones mask, same shape
         dcsr = rb.radial_mask_build_dense(wl.n, wl.block)
         dnnz = rb.radial_csr_info(dcsr)["nnz"]
@@ -313,7 +346,7 @@ def run_ours(args, rank, world, local_rank):
 
     # ---- end to end through the public API with host buffers
     e2e = None
-    if rank == 0 and not args.quick:
+    if rank == 0 and not args.quick and local_heads > 0:
         hq, hk, hv = (t.cpu().pin_memory() for t in (q, k, v))
         hdo = do.cpu().pin_memory() if backward else None
         ho = torch.empty(q.shape, dtype=torch.bfloat16).pin_memory()
@@ -328,7 +361,8 @@ def run_ours(args, rank, world, local_rank):
             v.copy_(hv, non_blocking=True)
             if backward:
                 do.copy_(hdo, non_blocking=True)
-            rb.radial_attn_fwd(csr, q, k, v, o=o, lse=lse, stream=stream)
+            if step_kind != "bwd":
+                rb.radial_attn_fwd(csr, q, k, v, o=o, lse=lse, stream=stream)
             if backward:
                 rb.radial_attn_bwd(csr, do, q, k, v, o, lse, dq, dk, dv, ws, stream=stream)
                 hdq.copy_(dq, non_blocking=True)
@@ -350,7 +384,8 @@ def run_ours(args, rank, world, local_rank):
         elt = q.numel() * 2
         h2d = 3 * elt + (elt if backward else 0)
         d2h = elt + lse.numel() * 4 + (3 * elt if backward else 0)
-        e2e = {"value": flops_step / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": e2e_ms,
+        e2e = {"value": (flops_step if not heads_mode else flops_step * wl.heads / local_heads) / (e2e_ms * 1e-3) / 1e12,
+               "unit": "TFLOP/s", "ms_per_step": e2e_ms,
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
                "path": "pinned host -> device copies, radial_attn_fwd%s via the C ABI, device -> host result copies"
                        % ("/bwd" if backward else "")}
@@ -373,15 +408,17 @@ def run_ours(args, rank, world, local_rank):
                 traffic = None
         line = {
             "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": ms_max, "higher_is_better": True, "scaling": "weak",
+            "warmup": args.warmup, "ms_per_step": ms_max, "higher_is_better": True,
+            "scaling": "strong" if heads_mode else "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded N(0,1) bf16 Q,K,V%s)" % (",dO" if backward else ""),
-            "config": config_of(wl, nnz),
+            "config": dict(config_of(wl, nnz), parallelism=(f"heads/{world}" if heads_mode else f"replica x{world}"),
+                           heads_per_rank_max=-(-wl.heads // world) if heads_mode else wl.heads),
             "pct_of_tensor_peak": 100.0 * value / world / peak,
             "mask_build_ms": mask_ms,
             "roofline": {"bound": "tensor", "kernel": fwd_kernel_name(), "achieved": fwd_tf, "peak": peak,
                          "unit": "TFLOP/s", "frac": fwd_tf / peak, "peak_source": f"{peak_src} bf16 burst",
                          "frac_of_sustained": fwd_tf / peak_sus, "traffic": traffic,
-                         "algorithmic_flops_per_launch": tile_flops(wl, nnz), "launch_ms": fwd_ms},
+                         "algorithmic_flops_per_launch": tile_flops(wl, nnz, heads=local_heads), "launch_ms": fwd_ms},
             "cpu_baseline": cpu,
             "e2e": e2e,
             "gpu_launches": int(launches),
@@ -497,6 +534,7 @@ def run_reference(args, rank, world):
     from oracle import mask as M
 
     wl = I.WORKLOADS[args.workload]
+    heads_mode = args.shard == "heads"
     st = M.tile_states_intervals(wl.frames, wl.tokens_per_frame, wl.block, True)
     nnz = int((st != 0).sum())
     # one head's K, V drawn on the CPU with the same recipe's generator
@@ -526,7 +564,8 @@ def run_reference(args, rank, world):
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": full_s * 1e3, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": config_of(wl, nnz),
+            "config": dict(config_of(wl, nnz), parallelism=(f"heads/{world}" if heads_mode else f"replica x{world}"),
+                           heads_per_rank_max=-(-wl.heads // world) if heads_mode else wl.heads),
             "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": _cores(), "kind": "oracle", "sample": sample},
             "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -547,6 +586,10 @@ def main():
     ap.add_argument("--sweep", action="store_true", help="add the frame-count scaling sweep (radial vs dense)")
     ap.add_argument("--lora", action="store_true", help="add one LoRA-adapted attention layer step (fwd+bwd)")
     ap.add_argument("--lora-rank", type=int, default=64)
+    ap.add_argument("--step", default=None, choices=["fwd", "bwd", "fwdbwd"],
+                    help="what one step runs (default: the workload's own: forward, or forward+backward)")
+    ap.add_argument("--shard", default="heads", choices=["heads", "replica"],
+                    help="multi-GPU: split the problem's heads across ranks (default) or run one replica per rank")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         args.warmup = 3
