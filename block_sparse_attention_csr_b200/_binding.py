@@ -17,7 +17,9 @@ import numpy as np
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_NAME = "libradial.so"
-lib_path = os.path.join(_HERE, LIB_NAME)
+# RADIAL_LIBRARY names another build of the same library (for instance the
+# bounds-checking libradial_debug.so); by default the in-tree release build.
+lib_path = os.environ.get("RADIAL_LIBRARY") or os.path.join(_HERE, LIB_NAME)
 
 RADIAL_OK = 0
 STATUS_NAMES = {0: "RADIAL_OK", 1: "RADIAL_EINVAL", 2: "RADIAL_EUNSUPPORTED", 3: "RADIAL_ENOMEM",
@@ -71,7 +73,7 @@ def load(path=None):
             return _lib
         p = path or lib_path
         if not os.path.exists(p):
-            raise RuntimeError(f"{LIB_NAME} not built at {p}; run block_sparse_attention_csr_b200.build")
+            raise RuntimeError(f"{os.path.basename(p)} not built at {p}; run block_sparse_attention_csr_b200.build")
         L = ctypes.CDLL(p)
         vp, i32, i64, sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t
         L.radial_params_default.argtypes = [ctypes.POINTER(radial_params)]

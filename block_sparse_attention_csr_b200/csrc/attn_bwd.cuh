@@ -215,7 +215,7 @@ __global__ void __launch_bounds__(384, 1)
       uint32_t it = 0, item_i = 0;
       for (int item = blockIdx.x; item < p.items; item += gridDim.x, ++item_i) {
         const int bh = item / p.nt;
-        const int u = p.col_order ? p.col_order[item - bh * p.nt] : item - bh * p.nt;
+        const int u = p.col_order ? RADIAL_CHECK_INDEX(p.col_order[item - bh * p.nt], 0, p.nt) : item - bh * p.nt;
         const int b = bh / p.heads, h = bh - b * p.heads;
         if (item_i > 0) mbar_wait(&bars->fix_empty, (item_i - 1) & 1, abort_flag);
         mbar_arrive_expect_tx(&bars->fix_full, 2 * C::TILE_BYTES);
@@ -225,7 +225,7 @@ __global__ void __launch_bounds__(384, 1)
           tma_load_4d(sV + x * 16384, &tmV, &bars->fix_full, x * 64, u * 128, h, b);
         }
         for (int q = p.col_ptr[u]; q < p.col_ptr[u + 1]; ++q, ++it) {
-          const int t = p.row_idx[q];
+          const int t = RADIAL_CHECK_INDEX(p.row_idx[q], 0, p.nt);
           const uint32_t st = it % C::STAGES, use = it / C::STAGES;
           if (use > 0) mbar_wait(&bars->st_empty[st], (use - 1) & 1, abort_flag);
           uint8_t* dstQ = sQ + st * 2 * C::TILE_BYTES;
@@ -254,7 +254,7 @@ __global__ void __launch_bounds__(384, 1)
       uint32_t it = 0, item_i = 0;
       for (int item = blockIdx.x; item < p.items; item += gridDim.x, ++item_i) {
         const int bh = item / p.nt;
-        const int u = p.col_order ? p.col_order[item - bh * p.nt] : item - bh * p.nt;
+        const int u = p.col_order ? RADIAL_CHECK_INDEX(p.col_order[item - bh * p.nt], 0, p.nt) : item - bh * p.nt;
         const uint32_t n_tiles = static_cast<uint32_t>(p.col_ptr[u + 1] - p.col_ptr[u]);
         mbar_wait(&bars->fix_full, item_i & 1, abort_flag);
         tc_fence_after();
@@ -326,7 +326,7 @@ __global__ void __launch_bounds__(384, 1)
     uint32_t it = 0, item_i = 0;
     for (int item = blockIdx.x; item < p.items; item += gridDim.x, ++item_i) {
       const int bh = item / p.nt;
-      const int u = p.col_order ? p.col_order[item - bh * p.nt] : item - bh * p.nt;
+      const int u = p.col_order ? RADIAL_CHECK_INDEX(p.col_order[item - bh * p.nt], 0, p.nt) : item - bh * p.nt;
       const int b = bh / p.heads, h = bh - b * p.heads;
       const int key = u * 128 + row;
       const bool valid = key < p.n;
@@ -338,7 +338,7 @@ __global__ void __launch_bounds__(384, 1)
       const float* dr_bh = p.dr + static_cast<int64_t>(bh) * p.n;
       for (uint32_t j = 0; j < n_tiles; ++j) {
         const uint32_t g = it + j;
-        const int t = p.row_idx[c0 + j];
+        const int t = RADIAL_CHECK_INDEX(p.row_idx[c0 + j], 0, p.nt);
         const bool partial = p.kind_t[c0 + j] != kTileFull;
         // this warpgroup's 64 queries: lse2 and dr -> shared memory
         float* vbuf = my_vec + (g & 1) * 128;
@@ -516,7 +516,7 @@ __global__ void __launch_bounds__(384, 1)
       uint32_t it = 0, item_i = 0;
       for (int item = blockIdx.x; item < p.items; item += gridDim.x, ++item_i) {
         const int bh = item / p.nt;
-        const int t = p.row_order ? p.row_order[item - bh * p.nt] : item - bh * p.nt;
+        const int t = p.row_order ? RADIAL_CHECK_INDEX(p.row_order[item - bh * p.nt], 0, p.nt) : item - bh * p.nt;
         const int b = bh / p.heads, h = bh - b * p.heads;
         if (item_i > 0) mbar_wait(&bars->fix_empty, (item_i - 1) & 1, abort_flag);
         mbar_arrive_expect_tx(&bars->fix_full, 2 * C::TILE_BYTES);
@@ -526,7 +526,7 @@ __global__ void __launch_bounds__(384, 1)
           tma_load_4d(sdO + x * 16384, &tmdO, &bars->fix_full, x * 64, t * 128, h, b);
         }
         for (int q = p.row_ptr[t]; q < p.row_ptr[t + 1]; ++q, ++it) {
-          const int kb = p.col_idx[q];
+          const int kb = RADIAL_CHECK_INDEX(p.col_idx[q], 0, p.nt);
           const uint32_t st = it % C::STAGES, use = it / C::STAGES;
           if (use > 0) mbar_wait(&bars->st_empty[st], (use - 1) & 1, abort_flag);
           uint8_t* dK = sK + st * 2 * C::TILE_BYTES;
@@ -567,7 +567,7 @@ __global__ void __launch_bounds__(384, 1)
       };
       for (int item = blockIdx.x; item < p.items; item += gridDim.x, ++item_i) {
         const int bh = item / p.nt;
-        const int t = p.row_order ? p.row_order[item - bh * p.nt] : item - bh * p.nt;
+        const int t = p.row_order ? RADIAL_CHECK_INDEX(p.row_order[item - bh * p.nt], 0, p.nt) : item - bh * p.nt;
         const uint32_t n_tiles = static_cast<uint32_t>(p.row_ptr[t + 1] - p.row_ptr[t]);
         mbar_wait(&bars->fix_full, item_i & 1, abort_flag);
         tc_fence_after();
@@ -606,7 +606,7 @@ __global__ void __launch_bounds__(384, 1)
     uint32_t it = 0, item_i = 0;
     for (int item = blockIdx.x; item < p.items; item += gridDim.x, ++item_i) {
       const int bh = item / p.nt;
-      const int t = p.row_order ? p.row_order[item - bh * p.nt] : item - bh * p.nt;
+      const int t = p.row_order ? RADIAL_CHECK_INDEX(p.row_order[item - bh * p.nt], 0, p.nt) : item - bh * p.nt;
       const int b = bh / p.heads, h = bh - b * p.heads;
       const int a = t * 128 + row;
       const bool valid = a < p.n;
@@ -618,7 +618,7 @@ __global__ void __launch_bounds__(384, 1)
       const uint32_t n_tiles = static_cast<uint32_t>(p.row_ptr[t + 1] - p0);
       for (uint32_t j = 0; j < n_tiles; ++j) {
         const uint32_t g = it + j, db = g & 1;
-        const int kb = p.col_idx[p0 + j];
+        const int kb = RADIAL_CHECK_INDEX(p.col_idx[p0 + j], 0, p.nt);
         const bool partial = p.kind[p0 + j] != kTileFull;
         uint32_t mw[4] = {0xffffffffu, 0xffffffffu, 0xffffffffu, 0xffffffffu};
         if (partial) {

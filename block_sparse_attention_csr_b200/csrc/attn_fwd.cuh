@@ -232,7 +232,7 @@ __global__ void __launch_bounds__(384, 1)
       };
       for (int item = blockIdx.x; item < p.items; item += gridDim.x, ++item_i) {
         const int bh = item / p.nt;
-        const int t = p.order ? p.order[item - bh * p.nt] : item - bh * p.nt;
+        const int t = p.order ? RADIAL_CHECK_INDEX(p.order[item - bh * p.nt], 0, p.nt) : item - bh * p.nt;
         const int b = bh / p.heads, h = bh - b * p.heads;
         if (item_i > 0) mbar_wait(&bars->q_empty, (item_i - 1) & 1, abort_flag);
         mbar_arrive_expect_tx(&bars->q_full, C::TILE_BYTES);
@@ -241,10 +241,10 @@ __global__ void __launch_bounds__(384, 1)
           tma_load_4d(sQ + x * 16384, &tmQ, &bars->q_full, x * 64, t * 128, h, b);
         const int p0 = p.row_ptr[t], p1 = p.row_ptr[t + 1];
         // K runs two columns ahead of V (S_{j+2} is issued before PV_j)
-        for (int q = p0; q < p0 + 2 && q < p1; ++q) load_k(p.col_idx[q], h, b);
+        for (int q = p0; q < p0 + 2 && q < p1; ++q) load_k(RADIAL_CHECK_INDEX(p.col_idx[q], 0, p.nt), h, b);
         for (int q = p0; q < p1; ++q) {
-          if (q + 2 < p1) load_k(p.col_idx[q + 2], h, b);
-          load_v(p.col_idx[q], h, b);
+          if (q + 2 < p1) load_k(RADIAL_CHECK_INDEX(p.col_idx[q + 2], 0, p.nt), h, b);
+          load_v(RADIAL_CHECK_INDEX(p.col_idx[q], 0, p.nt), h, b);
         }
       }
       // Drain: every slot's last fill must have landed before the CTA exits.
@@ -298,7 +298,7 @@ __global__ void __launch_bounds__(384, 1)
       };
       for (int item = blockIdx.x; item < p.items; item += gridDim.x, ++item_i) {
         const int bh = item / p.nt;
-        const int t = p.order ? p.order[item - bh * p.nt] : item - bh * p.nt;
+        const int t = p.order ? RADIAL_CHECK_INDEX(p.order[item - bh * p.nt], 0, p.nt) : item - bh * p.nt;
         const uint32_t n = static_cast<uint32_t>(p.row_ptr[t + 1] - p.row_ptr[t]);
         mbar_wait(&bars->q_full, item_i & 1, abort_flag);
         tc_fence_after();
@@ -338,7 +338,7 @@ __global__ void __launch_bounds__(384, 1)
     uint32_t it = 0, item_i = 0;
     for (int item = blockIdx.x; item < p.items; item += gridDim.x, ++item_i) {
       const int bh = item / p.nt;
-      const int t = p.order ? p.order[item - bh * p.nt] : item - bh * p.nt;
+      const int t = p.order ? RADIAL_CHECK_INDEX(p.order[item - bh * p.nt], 0, p.nt) : item - bh * p.nt;
       const int b = bh / p.heads, h = bh - b * p.heads;
       const int a = t * 128 + row;
       const bool valid = a < p.n;
@@ -348,14 +348,14 @@ __global__ void __launch_bounds__(384, 1)
       const uint32_t n = static_cast<uint32_t>(p.row_ptr[t + 1] - p0);
       float m = -INFINITY;  // running max of scaled logits, log2 domain
       float l = 0.f;        // this warp's part of the running sum of exp2(logit - m)
-      int kb_next = p.col_idx[p0];
+      int kb_next = RADIAL_CHECK_INDEX(p.col_idx[p0], 0, p.nt);
       uint8_t kind_next = p.kind[p0];
       for (uint32_t j = 0; j < n; ++j) {
         const uint32_t g = it + j, sb = g & 1;
         const int kb = kb_next;
         const bool part = kind_next != kTileFull;
         if (j + 1 < n) {
-          kb_next = p.col_idx[p0 + j + 1];
+          kb_next = RADIAL_CHECK_INDEX(p.col_idx[p0 + j + 1], 0, p.nt);
           kind_next = p.kind[p0 + j + 1];
         }
         mbar_wait(&bars->s_full[sb], (g >> 1) & 1, abort_flag);

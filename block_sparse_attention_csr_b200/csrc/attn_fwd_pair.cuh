@@ -164,7 +164,7 @@ __global__ void __launch_bounds__(384, 1)
       };
       for (int item = blockIdx.x; item < p.items; item += gridDim.x, ++item_i) {
         const int bh = item / p.np;
-        const int pr = p.pair_order ? p.pair_order[item - bh * p.np] : item - bh * p.np;
+        const int pr = p.pair_order ? RADIAL_CHECK_INDEX(p.pair_order[item - bh * p.np], 0, p.np) : item - bh * p.np;
         const int b = bh / p.heads, h = bh - b * p.heads;
         const bool two = 2 * pr + 1 < p.nt;
         if (item_i > 0) mbar_wait(&bars->q_empty, (item_i - 1) & 1, abort_flag);
@@ -175,10 +175,10 @@ __global__ void __launch_bounds__(384, 1)
           if (two) tma_load_4d(sQ + C::TILE_BYTES + x * 16384, &tmQ, &bars->q_full, x * 64, (2 * pr + 1) * 128, h, b);
         }
         const int u0 = p.pair_ptr[pr], u1 = p.pair_ptr[pr + 1];
-        load_k(p.pair_col[u0], h, b);
+        load_k(RADIAL_CHECK_INDEX(p.pair_col[u0], 0, p.nt), h, b);
         for (int u = u0; u < u1; ++u) {
-          if (u + 1 < u1) load_k(p.pair_col[u + 1], h, b);
-          load_v(p.pair_col[u], h, b);
+          if (u + 1 < u1) load_k(RADIAL_CHECK_INDEX(p.pair_col[u + 1], 0, p.nt), h, b);
+          load_v(RADIAL_CHECK_INDEX(p.pair_col[u], 0, p.nt), h, b);
         }
       }
       for (uint32_t x = (kc > C::K_SLOTS ? kc - C::K_SLOTS : 0); x < kc; ++x)
@@ -205,7 +205,7 @@ __global__ void __launch_bounds__(384, 1)
       uint32_t icnt[2] = {0u, 0u};    // items completed per query tile
       for (int item = blockIdx.x; item < p.items; item += gridDim.x, ++item_i) {
         const int bh = item / p.np;
-        const int pr = p.pair_order ? p.pair_order[item - bh * p.np] : item - bh * p.np;
+        const int pr = p.pair_order ? RADIAL_CHECK_INDEX(p.pair_order[item - bh * p.np], 0, p.np) : item - bh * p.np;
         const int u0 = p.pair_ptr[pr], u1 = p.pair_ptr[pr + 1];
         mbar_wait(&bars->q_full, item_i & 1, abort_flag);
         tc_fence_after();
@@ -313,7 +313,7 @@ __global__ void __launch_bounds__(384, 1)
     uint32_t g[2] = {0u, 0u}, icnt[2] = {0u, 0u};
     for (int item = blockIdx.x; item < p.items; item += gridDim.x) {
       const int bh = item / p.np;
-      const int pr = p.pair_order ? p.pair_order[item - bh * p.np] : item - bh * p.np;
+      const int pr = p.pair_order ? RADIAL_CHECK_INDEX(p.pair_order[item - bh * p.np], 0, p.np) : item - bh * p.np;
       const int b = bh / p.heads, h = bh - b * p.heads;
       const bool two = 2 * pr + 1 < p.nt;
       const int u0 = p.pair_ptr[pr], u1 = p.pair_ptr[pr + 1];
@@ -329,13 +329,13 @@ __global__ void __launch_bounds__(384, 1)
         qk[ti] = valid[ti] ? a - qi[ti] * p.s : 0;
       }
       uint8_t fl_next = p.pair_flag[u0];
-      int kb_next = p.pair_col[u0];
+      int kb_next = RADIAL_CHECK_INDEX(p.pair_col[u0], 0, p.nt);
       for (int u = u0; u < u1; ++u) {
         const uint8_t fl = fl_next;
         const int kb = kb_next;
         if (u + 1 < u1) {
           fl_next = p.pair_flag[u + 1];
-          kb_next = p.pair_col[u + 1];
+          kb_next = RADIAL_CHECK_INDEX(p.pair_col[u + 1], 0, p.nt);
         }
 #pragma unroll
         for (int ti = 0; ti < 2; ++ti) {

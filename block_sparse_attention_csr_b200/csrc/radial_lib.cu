@@ -6,6 +6,7 @@
 // allocates the mask's arrays, encodes TMA descriptors and launches.
 #include <cuda.h>
 #include <cuda_runtime.h>
+#include <nvtx3/nvToolsExt.h>
 
 #include <atomic>
 #include <cmath>
@@ -21,6 +22,7 @@
 #include "attn_bwd.cuh"
 #include "attn_fwd.cuh"
 #include "attn_fwd_pair.cuh"
+#include "attn_fwd_cta2.cuh"
 #include "mask_build.cuh"
 #include "sm100_primitives.cuh"
 
@@ -83,6 +85,15 @@ radial_status fail(radial_status s, const char* fmt, ...) {
 
 inline cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
 
+// An NVTX range around each entry point, so that profiler timelines show the
+// library's calls by name (no cost unless a profiler is attached).
+struct NvtxRange {
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+  NvtxRange(const NvtxRange&) = delete;
+  NvtxRange& operator=(const NvtxRange&) = delete;
+};
+
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 int sm_count() {
@@ -111,16 +122,16 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// 4D map over a bf16 [B, H, N, D] tensor (D contiguous), 128-row x 64-column
-// boxes with the 128-byte swizzle; rows past N read as zeros.
-radial_status make_bhnd_map(CUtensorMap* map, const void* base, const radial_desc& d) {
+// 4D map over a bf16 [B, H, N, D] tensor (D contiguous), box_rows-row x
+// 64-column boxes with the 128-byte swizzle; rows past N read as zeros.
+radial_status make_bhnd_map(CUtensorMap* map, const void* base, const radial_desc& d, uint32_t box_rows = 128) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return fail(RADIAL_ECUDA, "cuTensorMapEncodeTiled unavailable");
   cuuint64_t dims[4] = {static_cast<cuuint64_t>(d.head_dim), static_cast<cuuint64_t>(d.n_tokens),
                         static_cast<cuuint64_t>(d.heads), static_cast<cuuint64_t>(d.batch)};
   cuuint64_t strides[3] = {static_cast<cuuint64_t>(d.stride_n) * 2, static_cast<cuuint64_t>(d.stride_h) * 2,
                            static_cast<cuuint64_t>(d.stride_b) * 2};
-  cuuint32_t box[4] = {64, 128, 1, 1};
+  cuuint32_t box[4] = {64, box_rows, 1, 1};
   cuuint32_t estr[4] = {1, 1, 1, 1};
   CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box,
                   estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -389,6 +400,7 @@ void radial_params_default(radial_params* p) {
 
 radial_status radial_mask_build(int32_t frames, int32_t tokens_per_frame, int32_t block,
                                 const radial_params* params, radial_csr** out, void* stream) {
+  NvtxRange nvtx_range("radial_mask_build");
   if (!out) return fail(RADIAL_EINVAL, "out is NULL");
   *out = nullptr;
   radial_params def;
@@ -414,6 +426,7 @@ radial_status radial_mask_build(int32_t frames, int32_t tokens_per_frame, int32_
 }
 
 radial_status radial_mask_build_dense(int32_t n_tokens, int32_t block, radial_csr** out, void* stream) {
+  NvtxRange nvtx_range("radial_mask_build_dense");
   if (!out) return fail(RADIAL_EINVAL, "out is NULL");
   *out = nullptr;
   if (n_tokens < 1) return fail(RADIAL_EINVAL, "n_tokens must be >= 1");
@@ -440,6 +453,7 @@ radial_status radial_csr_info(const radial_csr* c, radial_csr_info_t* info) {
 radial_status radial_csr_copy_to_host(const radial_csr* c, int32_t* row_ptr, int32_t* col_idx,
                                       uint8_t* kind, int32_t* col_ptr, int32_t* row_idx,
                                       uint8_t* kind_t, int32_t* row_order, int32_t* col_order) {
+  NvtxRange nvtx_range("radial_csr_copy_to_host");
   if (!c) return fail(RADIAL_EINVAL, "csr is NULL");
   const TileLists& L = c->user;
   const size_t nb = static_cast<size_t>(L.nb), nnz = static_cast<size_t>(L.nnz);
@@ -506,14 +520,44 @@ bool schedule_lpt() {
   return lpt;
 }
 
-// RADIAL_FWD_KERNEL=single selects the one-query-tile forward kernel; the
-// default is the two-tile (pair) kernel.
-bool fwd_single_tile() {
-  static const bool single = [] {
+// Forward kernel choice: 0 two tiles per CTA (default), 1 one tile per CTA,
+// 2 one tile per CTA with the MMA shared by a CTA pair (RADIAL_FWD_KERNEL =
+// pair | single | cta2).
+int fwd_kernel_choice() {
+  static const int k = [] {
     const char* e = std::getenv("RADIAL_FWD_KERNEL");
-    return e && std::strcmp(e, "single") == 0;
+    if (e && std::strcmp(e, "single") == 0) return 1;
+    if (e && std::strcmp(e, "cta2") == 0) return 2;
+    return 0;
   }();
-  return single;
+  return k;
+}
+
+// Number of 2-CTA clusters of the CTA-pair forward that fit on the device at
+// once (looked up once per device).
+int pair_clusters(int smem) {
+  static int cached[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return sm_count() / 2;
+  if (cached[dev] > 0) return cached[dev];
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * (sm_count() / 2), 1, 1);
+  cfg.blockDim = dim3(384, 1, 1);
+  cfg.dynamicSmemBytes = static_cast<size_t>(smem);
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, radial_fwd_cta2_kernel<128>, &cfg) != cudaSuccess || n <= 0) {
+    cudaGetLastError();
+    n = sm_count() / 2;
+  }
+  cached[dev] = n;
+  return n;
 }
 
 template <int D>
@@ -549,6 +593,43 @@ radial_status launch_fwd_pair(const radial_csr* c, const radial_desc* d, const v
   const int grid = p.items < sm_count() ? p.items : sm_count();
   RADIAL_CUDA(cudaFuncSetAttribute(radial_fwd_pair_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
   radial_fwd_pair_kernel<D><<<grid, 384, smem, st>>>(mq, mk, mv, p);
+  RADIAL_LAUNCHED();
+  return RADIAL_OK;
+}
+
+radial_status launch_fwd_cta2(const radial_csr* c, const radial_desc* d, const void* q, const void* k,
+                              const void* v, void* o, float* lse, cudaStream_t st) {
+  CUtensorMap mq, mk, mv;
+  radial_status rs;
+  if ((rs = make_bhnd_map(&mq, q, *d)) != RADIAL_OK) return rs;
+  if ((rs = make_bhnd_map(&mk, k, *d, 64)) != RADIAL_OK) return rs;   // a CTA loads 64 keys of a tile
+  if ((rs = make_bhnd_map(&mv, v, *d)) != RADIAL_OK) return rs;       // and 64 columns of its values
+  FwdPairParams p;
+  p.pair_ptr = c->pairs.ptr;
+  p.pair_col = c->pairs.col;
+  p.pair_flag = c->pairs.flag;
+  p.pair_order = schedule_lpt() ? c->pairs.order : nullptr;
+  p.hd = c->hd;
+  p.cd = c->cd;
+  p.np = c->pairs.np;
+  p.nt = c->plan.nb;
+  p.f = c->f;
+  p.s = c->s;
+  p.n = c->n;
+  p.sink = c->sink;
+  p.heads = d->heads;
+  p.items = d->batch * d->heads * c->pairs.np;
+  p.o_sb = d->stride_b;
+  p.o_sh = d->stride_h;
+  p.o_sn = d->stride_n;
+  p.o = reinterpret_cast<__nv_bfloat16*>(o);
+  p.lse = lse;
+  p.scale_log2 = softmax_scale(d) * 1.4426950408889634f;
+  const int smem = FwdCta2Cfg<128>::SMEM_BYTES;
+  RADIAL_CUDA(cudaFuncSetAttribute(radial_fwd_cta2_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
+  const int clusters = pair_clusters(smem);
+  const int grid = 2 * (p.items < clusters ? p.items : clusters);
+  radial_fwd_cta2_kernel<128><<<grid, 384, smem, st>>>(mq, mk, mv, p);
   RADIAL_LAUNCHED();
   return RADIAL_OK;
 }
@@ -656,12 +737,15 @@ extern "C" {
 
 radial_status radial_attn_fwd(const radial_csr* c, const radial_desc* d, const void* q, const void* k,
                               const void* v, void* o, float* lse, void* stream) {
+  NvtxRange nvtx_range("radial_attn_fwd");
   radial_status rs = check_desc(c, d);
   if (rs != RADIAL_OK) return rs;
   if (!q || !k || !v || !o || !lse) return fail(RADIAL_EINVAL, "NULL tensor pointer");
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
     return fail(RADIAL_EINVAL, "tensor pointers must be 16-byte aligned");
-  if (!fwd_single_tile()) {
+  const int choice = fwd_kernel_choice();
+  if (choice == 2 && d->head_dim == 128) return launch_fwd_cta2(c, d, q, k, v, o, lse, as_stream(stream));
+  if (choice != 1) {
     if (d->head_dim == 128) return launch_fwd_pair<128>(c, d, q, k, v, o, lse, as_stream(stream));
     return launch_fwd_pair<64>(c, d, q, k, v, o, lse, as_stream(stream));
   }
@@ -678,6 +762,7 @@ size_t radial_attn_bwd_workspace_size(const radial_desc* d) {
 radial_status radial_attn_bwd(const radial_csr* c, const radial_desc* d, const void* dout, const void* q,
                               const void* k, const void* v, const void* o, const float* lse, void* dq,
                               void* dk, void* dv, void* workspace, size_t workspace_bytes, void* stream) {
+  NvtxRange nvtx_range("radial_attn_bwd");
   radial_status rs = check_desc(c, d);
   if (rs != RADIAL_OK) return rs;
   if (!dout || !q || !k || !v || !o || !lse || !dq || !dk || !dv || !workspace)
@@ -738,6 +823,7 @@ extern "C" {
 radial_status radial_attn_bwd_noalloc(const radial_csr* c, const radial_desc* d, const void* dout,
                                       const void* q, const void* k, const void* v, const void* o,
                                       const float* lse, void* dq, void* dk, void* dv, void* stream) {
+  NvtxRange nvtx_range("radial_attn_bwd_noalloc");
   radial_status rs = check_desc(c, d);
   if (rs != RADIAL_OK) return rs;
   if (!dout || !q || !k || !v || !o || !lse || !dq || !dk || !dv)
@@ -759,12 +845,15 @@ radial_status radial_attn_bwd_noalloc(const radial_csr* c, const radial_desc* d,
 }
 
 radial_status radial_device_status(void* stream) {
+  NvtxRange nvtx_range("radial_device_status");
   RADIAL_CUDA(cudaStreamSynchronize(as_stream(stream)));
   int flag = 0;
   RADIAL_CUDA(cudaMemcpyFromSymbol(&flag, g_device_error, sizeof(int)));
   if (flag != 0) {
     const int zero = 0;
     RADIAL_CUDA(cudaMemcpyToSymbol(g_device_error, &zero, sizeof(int)));
+    if (flag == kErrBounds)
+      return fail(RADIAL_EDEVICE, "a kernel read an out-of-range index from the mask's arrays (code %d)", flag);
     return fail(RADIAL_EDEVICE, "a kernel aborted after a bounded wait ran out (code %d)", flag);
   }
   RADIAL_CUDA(cudaGetLastError());

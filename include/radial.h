@@ -47,7 +47,9 @@ typedef enum radial_status {
   RADIAL_EUNSUPPORTED = 2,  /* well-formed but outside what the kernels implement */
   RADIAL_ENOMEM = 3,        /* a device or host allocation failed */
   RADIAL_ECUDA = 4,         /* a CUDA runtime or driver call failed */
-  RADIAL_EDEVICE = 5        /* a kernel aborted after a bounded wait ran out */
+  RADIAL_EDEVICE = 5        /* a kernel aborted after a bounded wait ran out (or, in
+                               the bounds-checking debug build, read an out-of-range
+                               index from the mask's arrays) */
 } radial_status;
 
 /* Mask parameters.  sink: 1 = every query also attends to all tokens of frame

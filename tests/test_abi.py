@@ -98,3 +98,12 @@ def test_bwd_workspace_size(lib):
 
 def test_csr_free_null_is_noop(lib):
     lib.radial_csr_free(None)
+
+
+def test_debug_build_exports_the_same_symbols(lib):
+    """libradial_debug.so (-DRADIAL_DEBUG: device-side range checks of every
+    index read from the mask's arrays) is the same ABI."""
+    assert os.path.exists(build_mod.OUT_DEBUG)
+    dbg = ctypes.CDLL(build_mod.OUT_DEBUG)
+    for n in _declared_functions():
+        assert hasattr(dbg, n), n
