@@ -181,6 +181,91 @@ def sample_rows(n, count, s, B, seed):
     return np.sort(np.concatenate([fixed, extra]))
 
 
+def sample_runs(n, count, s, B, seed, run=64):
+    """Seeded sample of about `count` query rows made of runs of `run`
+    consecutive rows: the first and last rows, the tail block, a run across
+    each of a random half-budget of frame boundaries, and random runs for the
+    rest -- sorted, unique.  Runs let forward_runs / dq_runs evaluate many
+    rows against one key superset."""
+    rng = np.random.default_rng(seed)
+    n_runs = max(1, count // run)
+    starts = [0, max(0, n - run)]
+    tail0 = (n // B) * B
+    if tail0 < n:
+        starts.append(tail0)
+    bounds = np.arange(s, n, s, dtype=np.int64)
+    if bounds.size:
+        take = min(bounds.size, max(0, n_runs // 2))
+        pick = rng.choice(bounds, size=take, replace=False) if take else np.zeros(0, np.int64)
+        starts += [int(b) - run // 2 for b in pick]
+    while len(starts) < n_runs:
+        starts.append(int(rng.integers(0, max(1, n - run + 1))))
+    rows = np.concatenate([np.arange(max(0, a), min(n, a + run), dtype=np.int64) for a in starts])
+    return np.unique(rows)
+
+
+def _runs_in_frames(rows, s, max_run):
+    """Split sorted unique rows into [a0, a1) runs of consecutive rows inside
+    one frame, at most max_run long."""
+    rows = np.asarray(rows, dtype=np.int64)
+    out = []
+    i = 0
+    while i < rows.size:
+        a0 = int(rows[i])
+        j = i + 1
+        while (j < rows.size and rows[j] == rows[j - 1] + 1 and rows[j] // s == a0 // s
+               and j - i < max_run):
+            j += 1
+        out.append((i, j, a0, int(rows[j - 1]) + 1))
+        i = j
+    return out
+
+
+def forward_runs(q, k, v, rows, f, s, sink=True, scale=None, max_run=128, spec=None):
+    """O and LSE of the given sorted query rows of one (batch, head): Eq.2
+    evaluated for each run of consecutive rows of one frame against the run's
+    key superset (mask.key_superset: every key it leaves out is masked for
+    each row of the run, and adds exp(-inf) = 0).  Returns (O_rows, LSE_rows)."""
+    k, v = _as64(k), _as64(v)
+    rows = np.asarray(rows, dtype=np.int64)
+    scale = 1.0 / np.sqrt(k.shape[1]) if scale is None else scale
+    O = np.empty((rows.size, k.shape[1]))
+    L = np.empty(rows.size)
+    for i0, i1, a0, a1 in _runs_in_frames(rows, s, max_run):
+        keys = _mask.key_superset(a0, a1, f, s, sink, spec)
+        r = rows[i0:i1]
+        S = (_as64(q[r]) @ k[keys].T) * scale
+        S = np.where(_mask.pair_mask(r, keys, f, s, sink, spec), S, -np.inf)
+        m = S.max(axis=1, keepdims=True)
+        P = np.exp(S - m)
+        l = P.sum(axis=1, keepdims=True)
+        O[i0:i1] = (P @ v[keys]) / l
+        L[i0:i1] = m[:, 0] + np.log(l[:, 0])
+    return O, L
+
+
+def dq_runs(q, k, v, do, rows, f, s, sink=True, scale=None, max_run=128, spec=None):
+    """dQ of the given sorted query rows of one (batch, head), run by run as
+    forward_runs (each row's O, LSE and rowsum(dO o O) recomputed in fp64)."""
+    k, v = _as64(k), _as64(v)
+    rows = np.asarray(rows, dtype=np.int64)
+    scale = 1.0 / np.sqrt(k.shape[1]) if scale is None else scale
+    out = np.empty((rows.size, k.shape[1]))
+    for i0, i1, a0, a1 in _runs_in_frames(rows, s, max_run):
+        keys = _mask.key_superset(a0, a1, f, s, sink, spec)
+        r = rows[i0:i1]
+        kk, vv = k[keys], v[keys]
+        S = np.where(_mask.pair_mask(r, keys, f, s, sink, spec), (_as64(q[r]) @ kk.T) * scale, -np.inf)
+        m = S.max(axis=1, keepdims=True)
+        P = np.exp(S - m)
+        P /= P.sum(axis=1, keepdims=True)
+        dor = _as64(do[r])
+        o = P @ vv
+        dS = P * (dor @ vv.T - (dor * o).sum(axis=1)[:, None])
+        out[i0:i1] = scale * (dS @ kk)
+    return out
+
+
 # ---------------------------------------------------------------------------
 # Whole-head statistics and key-column gradients (dK, dV at large shapes)
 # ---------------------------------------------------------------------------
@@ -218,12 +303,14 @@ def head_row_stats(q, k, v, do, f, s, sink=True, scale=None, chunk=128, threads=
         a0, a1 = rng
         keys = _mask.key_superset(a0, a1, f, s, sink, spec)
         rows = np.arange(a0, a1, dtype=np.int64)
-        S = (q[a0:a1] @ k[keys].T) * scale
-        S = np.where(_mask.pair_mask(rows, keys, f, s, sink, spec), S, -np.inf)
+        S = q[a0:a1] @ k[keys].T
+        S *= scale
+        np.copyto(S, -np.inf, where=~_mask.pair_mask(rows, keys, f, s, sink, spec))
         m = S.max(axis=1, keepdims=True)
-        P = np.exp(S - m)
-        l = P.sum(axis=1, keepdims=True)
-        o = (P @ v[keys]) / l
+        S -= m
+        np.exp(S, out=S)                       # S now holds P = exp(S - m)
+        l = S.sum(axis=1, keepdims=True)
+        o = (S @ v[keys]) / l
         lse[a0:a1] = m[:, 0] + np.log(l[:, 0])
         dr[a0:a1] = (do[a0:a1] * o).sum(axis=1)
 

@@ -42,6 +42,26 @@ def _dq_rows(args):
     return A.dq_rows(q, k, v, do, rows, f, s, sink, scale)
 
 
+def _fwd_runs(args):
+    from oracle import attention as A
+    q_rows, k, v, rows, f, s, sink, scale = args
+    n = k.shape[0]
+    q = np.zeros((n, k.shape[1]))
+    q[rows] = q_rows
+    return A.forward_runs(q, k, v, rows, f, s, sink, scale)
+
+
+def _dq_runs(args):
+    from oracle import attention as A
+    q_rows, k, v, do_rows, rows, f, s, sink, scale = args
+    n = k.shape[0]
+    q = np.zeros((n, k.shape[1]))
+    do = np.zeros((n, k.shape[1]))
+    q[rows] = q_rows
+    do[rows] = do_rows
+    return A.dq_runs(q, k, v, do, rows, f, s, sink, scale)
+
+
 def _bwd_head(args):
     """Forward and backward of one whole (batch, head) by the dense reference."""
     from oracle import attention as A
@@ -61,7 +81,8 @@ def cores():
 
 
 def run(fn_name, tasks, workers=None):
-    fn = {"fwd_rows": _fwd_rows, "dq_rows": _dq_rows, "bwd_head": _bwd_head}[fn_name]
+    fn = {"fwd_rows": _fwd_rows, "dq_rows": _dq_rows, "fwd_runs": _fwd_runs, "dq_runs": _dq_runs,
+          "bwd_head": _bwd_head}[fn_name]
     if not tasks:
         return []
     c = cores()

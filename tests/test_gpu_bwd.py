@@ -138,13 +138,13 @@ def _large_check(name, rows_per_head, dkdv_heads, cols_per_head):
     # sampled dQ rows against the reference, every head
     tasks, got = [], []
     for h in range(wl.heads):
-        rows = A.sample_rows(wl.n, rows_per_head, wl.tokens_per_frame, wl.block, seed=2000 + h)
+        rows = A.sample_runs(wl.n, rows_per_head, wl.tokens_per_frame, wl.block, seed=2000 + h)
         ridx = torch.as_tensor(rows, device=DEV)
         tasks.append((q[0, h, ridx].double().cpu().numpy(), k[0, h].float().cpu().numpy(),
                       v[0, h].float().cpu().numpy(), do[0, h, ridx].double().cpu().numpy(),
                       rows, wl.frames, wl.tokens_per_frame, True, scale))
         got.append(dq[0, h, ridx].float().cpu().numpy())
-    ref = oracle_pool.run("dq_rows", tasks)
+    ref = oracle_pool.run("dq_runs", tasks)
     err = max(np.abs(g - r).max() for g, r in zip(got, ref))
     assert err <= G_MAX, f"{name}: dQ max-abs {err:.3e}"
 

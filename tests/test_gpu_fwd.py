@@ -119,13 +119,13 @@ def _sampled_check(name, rows_per_head, heads=None):
     tasks, keep = [], []
     scale = 1.0 / np.sqrt(wl.head_dim)
     for h in heads:
-        rows = A.sample_rows(n, rows_per_head, wl.tokens_per_frame, wl.block, seed=1000 + h)
+        rows = A.sample_runs(n, rows_per_head, wl.tokens_per_frame, wl.block, seed=1000 + h)
         ridx = torch.as_tensor(rows, device=DEV)
         tasks.append((q[0, h, ridx].float().cpu().numpy().astype(np.float64),
                       k[0, h].float().cpu().numpy(), v[0, h].float().cpu().numpy(),
                       rows, wl.frames, wl.tokens_per_frame, True, scale))
         keep.append((o[0, h, ridx].float().cpu().numpy(), lse[0, h, ridx].cpu().numpy()))
-    res = oracle_pool.run("fwd_rows", tasks)
+    res = oracle_pool.run("fwd_runs", tasks)
     o_g = np.concatenate([a for a, _ in keep])
     l_g = np.concatenate([b for _, b in keep])
     o_r = np.concatenate([a for a, _ in res])

@@ -66,3 +66,33 @@ def test_dkdv_cols_planted_wrong_statistics_fail():
     dk, _ = A.dkdv_cols(q, k, v, do, lse, dr, cols, f, s, True)
     dk_bad, _ = A.dkdv_cols(q, k, v, do, lse, np.roll(dr, 1), cols, f, s, True)
     assert np.abs(dk - dk_bad).max() > 1e-3
+
+
+@pytest.mark.parametrize("f,s,sink,seed", [(9, 30, True, 1), (40, 3, True, 2), (64, 4, False, 3),
+                                           (6, 50, False, 4), (12, 17, True, 5)])
+def test_forward_runs_and_dq_runs_equal_dense(f, s, sink, seed):
+    rng = np.random.default_rng(seed)
+    n, d = f * s, 16
+    q, k, v, do = (rng.standard_normal((n, d)) for _ in range(4))
+    scale = 1.0 / np.sqrt(d)
+    allowed = M.token_mask(f, s, sink)
+    o, lse = A.forward(q, k, v, allowed, scale)
+    dq, _, _ = A.backward(q, k, v, o, do, lse, allowed, scale)
+    rows = A.sample_runs(n, 60, s, 16, seed=seed, run=8)
+    o2, l2 = A.forward_runs(q, k, v, rows, f, s, sink, max_run=5)
+    np.testing.assert_allclose(o2, o[rows], rtol=0, atol=1e-12)
+    np.testing.assert_allclose(l2, lse[rows], rtol=0, atol=1e-12)
+    np.testing.assert_allclose(A.dq_runs(q, k, v, do, rows, f, s, sink, max_run=5), dq[rows], rtol=0, atol=1e-12)
+
+
+def test_sample_runs_cover_the_edges():
+    f, s, B = 20, 50, 16
+    n = f * s
+    rows = A.sample_runs(n, 400, s, B, seed=0, run=16)
+    assert np.all(np.diff(rows) > 0) and rows[0] == 0 and rows[-1] == n - 1
+    tail0 = (n // B) * B
+    assert np.isin(np.arange(tail0, n), rows).all()
+    # runs that straddle frame boundaries
+    straddle = [b for b in range(s, n, s) if b - 1 in rows and b in rows]
+    assert len(straddle) >= 5
+    assert 300 <= rows.size <= 520
