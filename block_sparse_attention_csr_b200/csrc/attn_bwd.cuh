@@ -336,28 +336,18 @@ __global__ void __launch_bounds__(384, 1)
       const uint32_t n_tiles = static_cast<uint32_t>(p.col_ptr[u + 1] - c0);
       const float* lse_bh = p.lse + static_cast<int64_t>(bh) * p.n;
       const float* dr_bh = p.dr + static_cast<int64_t>(bh) * p.n;
-      // This thread's slot of a query tile's row statistics: lse2 (rows 0-63)
-      // or dr (rows 64-127) of query 64 wg + (row & 63).
-      auto vec_of = [&](int t) {
-        const int a = t * 128 + 64 * wg + (row & 63);
-        if (row < 64) return a < p.n ? lse_bh[a] * kLog2e : INFINITY;
-        return a < p.n ? dr_bh[a] : 0.f;
-      };
-      // the next tile's index, kind and row statistics are fetched one tile
-      // ahead, so their global-memory latency hides behind the current tile
-      int t_next = RADIAL_CHECK_INDEX(p.row_idx[c0], 0, p.nt);
-      bool part_next = p.kind_t[c0] != kTileFull;
-      float v_next = vec_of(t_next);
       for (uint32_t j = 0; j < n_tiles; ++j) {
         const uint32_t g = it + j;
-        const int t = t_next;
-        const bool partial = part_next;
+        const int t = RADIAL_CHECK_INDEX(p.row_idx[c0 + j], 0, p.nt);
+        const bool partial = p.kind_t[c0 + j] != kTileFull;
         // this warpgroup's 64 queries: lse2 and dr -> shared memory
         float* vbuf = my_vec + (g & 1) * 128;
-        vbuf[row] = v_next;
-        if (j + 1 < n_tiles) {
-          t_next = RADIAL_CHECK_INDEX(p.row_idx[c0 + j + 1], 0, p.nt);
-          part_next = p.kind_t[c0 + j + 1] != kTileFull;
+        {
+          const int a = t * 128 + 64 * wg + (row & 63);
+          if (row < 64)
+            vbuf[row] = a < p.n ? lse_bh[a] * kLog2e : INFINITY;
+          else
+            vbuf[row] = a < p.n ? dr_bh[a] : 0.f;
         }
         named_bar_sync(1 + wg, 128);
         uint32_t mw[4] = {0xffffffffu, 0xffffffffu, 0xffffffffu, 0xffffffffu};
@@ -368,39 +358,34 @@ __global__ void __launch_bounds__(384, 1)
             mw[0] = mw[1] = mw[2] = mw[3] = 0u;
         }
         const uint32_t modes = partial ? chunk_modes(mw) : 0u;
-        const uint32_t mode0 = (modes >> (4 * wg)) & 3u, mode1 = (modes >> (4 * wg + 2)) & 3u;
-        // pass 1: P^T = exp2(S^T * scale*log2e - lse2), kept in fp32 for pass 2.
-        // Both 32-column chunks of S^T are loaded before one wait; pr holds S^T,
-        // then P^T (fp32 bits) in place.
+        // pass 1: P^T = exp2(S^T * scale*log2e - lse2), kept in fp32 for pass 2
         mbar_wait(&bars->s_full, g & 1, abort_flag);
         __syncwarp();
         tc_fence_after();
-        uint32_t pr[64];
-        if (mode0 != 2u) tmem_ld32(tmem + lane_addr + TM_S + (2 * wg) * 32, *reinterpret_cast<uint32_t(*)[32]>(&pr[0]));
-        if (mode1 != 2u)
-          tmem_ld32(tmem + lane_addr + TM_S + (2 * wg + 1) * 32, *reinterpret_cast<uint32_t(*)[32]>(&pr[32]));
-        tmem_wait_ld();
+        float pv[64];
 #pragma unroll
         for (int c = 0; c < 2; ++c) {
           const int gc = 2 * wg + c;  // 32-column chunk of the tile
-          const uint32_t mode = c == 0 ? mode0 : mode1;
+          const uint32_t mode = (modes >> (2 * gc)) & 3u;
           uint32_t pw[16];
           if (mode == 2u) {  // every lane of the warp masks this chunk: P^T = 0
 #pragma unroll
-            for (int e = 0; e < 32; ++e) pr[32 * c + e] = 0u;
+            for (int e = 0; e < 32; ++e) pv[32 * c + e] = 0.f;
 #pragma unroll
             for (int e = 0; e < 16; ++e) pw[e] = 0u;
           } else {
+            uint32_t rs[32];
+            tmem_ld32(tmem + lane_addr + TM_S + gc * 32, rs);
+            tmem_wait_ld();
             const uint32_t bits = mode == 0u ? 0xffffffffu : mw[gc];
 #pragma unroll
             for (int e = 0; e < 32; ++e) {
-              const float x = fmaf(__uint_as_float(pr[32 * c + e]), p.scale_log2, -vbuf[c * 32 + e]);
+              const float x = fmaf(__uint_as_float(rs[e]), p.scale_log2, -vbuf[c * 32 + e]);
               const float pe = ex2_approx(x);
-              pr[32 * c + e] = __float_as_uint((mode == 0u || ((bits >> e) & 1u)) ? pe : 0.f);
+              pv[32 * c + e] = (mode == 0u || ((bits >> e) & 1u)) ? pe : 0.f;
             }
 #pragma unroll
-            for (int e = 0; e < 16; ++e)
-              pw[e] = pack_bf16x2(__uint_as_float(pr[32 * c + 2 * e]), __uint_as_float(pr[32 * c + 2 * e + 1]));
+            for (int e = 0; e < 16; ++e) pw[e] = pack_bf16x2(pv[32 * c + 2 * e], pv[32 * c + 2 * e + 1]);
           }
           // bf16 P^T goes to this warpgroup's own columns, over S^T it has already read
           tmem_st16(tmem + lane_addr + TM_S + 64 * wg + c * 16, pw);
@@ -408,27 +393,27 @@ __global__ void __launch_bounds__(384, 1)
         tmem_wait_st();
         tc_fence_before();
         mbar_arrive(&bars->p_ready[g & 1]);
-        if (j + 1 < n_tiles) v_next = vec_of(t_next);  // consumed at the top of the next tile
-        // pass 2: dS^T = P^T * (dP^T - Dr), one 32-column chunk at a time
+        // pass 2: dS^T = P^T * (dP^T - Dr)
         mbar_wait(&bars->dp_full, g & 1, abort_flag);
         __syncwarp();
         tc_fence_after();
 #pragma unroll
         for (int c = 0; c < 2; ++c) {
-          const uint32_t mode = c == 0 ? mode0 : mode1;
+          const int gc = 2 * wg + c;
+          const uint32_t mode = (modes >> (2 * gc)) & 3u;
           uint32_t dw[16];
           if (mode == 2u) {
 #pragma unroll
             for (int e = 0; e < 16; ++e) dw[e] = 0u;
           } else {
             uint32_t rp[32];
-            tmem_ld32(tmem + lane_addr + TM_DP + (2 * wg + c) * 32, rp);
+            tmem_ld32(tmem + lane_addr + TM_DP + gc * 32, rp);
             tmem_wait_ld();
 #pragma unroll
             for (int e = 0; e < 16; ++e) {
               const int q0 = c * 32 + 2 * e;  // query index inside this warpgroup's 64
-              const float d0 = __uint_as_float(pr[q0]) * (__uint_as_float(rp[2 * e]) - vbuf[64 + q0]);
-              const float d1 = __uint_as_float(pr[q0 + 1]) * (__uint_as_float(rp[2 * e + 1]) - vbuf[64 + q0 + 1]);
+              const float d0 = pv[q0] * (__uint_as_float(rp[2 * e]) - vbuf[64 + q0]);
+              const float d1 = pv[q0 + 1] * (__uint_as_float(rp[2 * e + 1]) - vbuf[64 + q0 + 1]);
               dw[e] = pack_bf16x2(d0, d1);
             }
           }
@@ -631,28 +616,23 @@ __global__ void __launch_bounds__(384, 1)
       const float drow = valid ? p.dr[static_cast<int64_t>(bh) * p.n + a] : 0.f;
       const int p0 = p.row_ptr[t];
       const uint32_t n_tiles = static_cast<uint32_t>(p.row_ptr[t + 1] - p0);
-      FwdParams mp{};
-      mp.f = p.f;
-      mp.s = p.s;
-      mp.n = p.n;
-      mp.sink = p.sink;
-      mp.hd = p.hd;
-      mp.cd = p.cd;
-      // the next tile's column and kind are fetched one tile ahead
-      int kb_next = RADIAL_CHECK_INDEX(p.col_idx[p0], 0, p.nt);
-      bool part_next = p.kind[p0] != kTileFull;
       for (uint32_t j = 0; j < n_tiles; ++j) {
         const uint32_t g = it + j, db = g & 1;
-        const int kb = kb_next;
-        const bool partial = part_next;
-        if (j + 1 < n_tiles) {
-          kb_next = RADIAL_CHECK_INDEX(p.col_idx[p0 + j + 1], 0, p.nt);
-          part_next = p.kind[p0 + j + 1] != kTileFull;
-        }
+        const int kb = RADIAL_CHECK_INDEX(p.col_idx[p0 + j], 0, p.nt);
+        const bool partial = p.kind[p0 + j] != kTileFull;
         uint32_t mw[4] = {0xffffffffu, 0xffffffffu, 0xffffffffu, 0xffffffffu};
         if (partial) {
           mw[0] = mw[1] = mw[2] = mw[3] = 0u;
-          if (valid) row_mask_bits(mp, qi, qk, kb * 128, mw);
+          if (valid) {
+            FwdParams mp{};
+            mp.f = p.f;
+            mp.s = p.s;
+            mp.n = p.n;
+            mp.sink = p.sink;
+            mp.hd = p.hd;
+            mp.cd = p.cd;
+            row_mask_bits(mp, qi, qk, kb * 128, mw);
+          }
         }
         // dS buffer db was read by the dQ MMA of tile g-2
         if (g >= 2) {
@@ -660,18 +640,30 @@ __global__ void __launch_bounds__(384, 1)
           __syncwarp();
         }
         const uint32_t modes = partial ? chunk_modes(mw) : 0u;
-        const uint32_t mode0 = (modes >> (4 * wg)) & 3u, mode1 = (modes >> (4 * wg + 2)) & 3u;
         mbar_wait(&bars->s_full, g & 1, abort_flag);
         __syncwarp();
         tc_fence_after();
-        // dS = P o (dP - Dr) of one 32-column chunk -> bf16 in TMEM
-        auto chunk = [&](int c, uint32_t mode, const uint32_t(&rs)[32], const uint32_t(&rp)[32]) {
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
           const int gc = 2 * wg + c;
+          const uint32_t mode = (modes >> (2 * gc)) & 3u;
           uint32_t dw[16];
           if (mode == 2u) {  // every lane of the warp masks this chunk: dS = 0
 #pragma unroll
             for (int e = 0; e < 16; ++e) dw[e] = 0u;
+            if (c == 1) {  // S and dP fully read: the next tile's S / dP may overwrite them
+              tc_fence_before();
+              mbar_arrive(&bars->s_free);
+            }
           } else {
+            uint32_t rs[32], rp[32];
+            tmem_ld32(tmem + lane_addr + TM_S + gc * 32, rs);
+            tmem_ld32(tmem + lane_addr + TM_DP + gc * 32, rp);
+            tmem_wait_ld();
+            if (c == 1) {  // S and dP fully read: the next tile's S / dP may overwrite them
+              tc_fence_before();
+              mbar_arrive(&bars->s_free);
+            }
             const uint32_t bits = mw[gc];
 #pragma unroll
             for (int e = 0; e < 16; ++e) {
@@ -686,21 +678,6 @@ __global__ void __launch_bounds__(384, 1)
             }
           }
           tmem_st16(tmem + lane_addr + TM_DS + db * 64 + gc * 16, dw);
-        };
-#pragma unroll
-        for (int c = 0; c < 2; ++c) {
-          const uint32_t mode = c == 0 ? mode0 : mode1;
-          uint32_t rs[32], rp[32];
-          if (mode != 2u) {
-            tmem_ld32(tmem + lane_addr + TM_S + (2 * wg + c) * 32, rs);
-            tmem_ld32(tmem + lane_addr + TM_DP + (2 * wg + c) * 32, rp);
-            tmem_wait_ld();
-          }
-          if (c == 1) {  // S and dP fully read: the next tile's S / dP may overwrite them
-            tc_fence_before();
-            mbar_arrive(&bars->s_free);
-          }
-          chunk(c, mode, rs, rp);
         }
         tmem_wait_st();
         tc_fence_before();
