@@ -289,26 +289,21 @@ __device__ __forceinline__ uint32_t mapa_shared(uint32_t local_addr, uint32_t ra
   return r;
 }
 
-// Arrive (release, cluster scope) on an mbarrier named by a shared::cluster
-// address, possibly in the other CTA of the pair.
+// Arrive on an mbarrier named by a shared::cluster address, possibly in the
+// other CTA of the pair.  The default (release, CTA scope) semantics are
+// enough: what a remote arrival publishes is TMEM state, ordered by the
+// tcgen05 fences around it, not ordinary memory; a cluster-scope release
+// would fence every arrival.
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
-  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+  asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
 }
 
 __device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t* bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.b32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity)
-      : "memory");
-  return ok != 0;
+  return mbar_try_wait(bar, parity);
 }
 
-// Bounded wait (as mbar_wait) with cluster-scope acquire: for barriers that
-// the other CTA of the pair arrives on.
+// Bounded wait (as mbar_wait) for barriers that the other CTA of the pair
+// arrives on.
 __device__ __forceinline__ bool mbar_wait_cl(uint64_t* bar, uint32_t parity, volatile int* abort) {
   if (mbar_try_wait_cluster(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
