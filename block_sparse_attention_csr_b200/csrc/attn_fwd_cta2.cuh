@@ -53,6 +53,13 @@
 
 namespace radial {
 
+// Exponential pairs of the softmax evaluated on the FMA pipe (exp2_fma_x2)
+// instead of the MUFU: bit e selects pair e of every 16-pair (32-key) chunk.
+#ifndef RADIAL_EXP2_FMA_PAIRS
+#define RADIAL_EXP2_FMA_PAIRS 0u
+#endif
+__host__ __device__ constexpr bool exp2_on_fma(int e) { return ((RADIAL_EXP2_FMA_PAIRS >> e) & 1u) != 0u; }
+
 template <int D>
 struct FwdCta2Cfg {
   static_assert(D == 128, "the CTA-pair forward is implemented for head_dim 128");
@@ -339,6 +346,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
       bool started = false;  // a column of this tile has been processed
       uint8_t fl_next = p.pair_flag[u0];
       int kb_next = RADIAL_CHECK_INDEX(p.pair_col[u0], 0, p.nt);
+      // S of the column being processed.  While a column's P is computed, the
+      // next column's S (already in the other S buffer) is loaded into the
+      // halves of r that P no longer needs, so the TMEM round trip of one
+      // column hides behind the exponentials of the previous one.
+      uint32_t r[64];
+      bool preloaded = false;
       for (uint32_t j = 0; j < n; ++j) {
         const uint32_t g = it + j, sb = g & 1;
         const uint8_t fl = fl_next;
@@ -348,10 +361,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
           kb_next = RADIAL_CHECK_INDEX(p.pair_col[u0 + j + 1], 0, p.nt);
         }
         const uint32_t tm_p = tmem + lane_addr + C::TM_P0 + sb * 64 + wg * 32;
-        checked(mbar_wait(&bars->s_full[sb], (g >> 1) & 1, abort_flag));
-        tc_fence_after();
         if (!(fl & in_bit)) {
           // the column belongs to the other tile only: S is not needed, P = 0
+          checked(mbar_wait(&bars->s_full[sb], (g >> 1) & 1, abort_flag));
+          tc_fence_after();
           warp_arrive(&bars->s_empty[sb]);
           if (g >= 2) {
             checked(mbar_wait(&bars->pv_done[sb], ((g >> 1) - 1) & 1, abort_flag));
@@ -366,10 +379,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
           warp_arrive(&bars->p_full[sb]);
           continue;
         }
-        const uint32_t tm_s = tmem + lane_addr + C::TM_S0 + sb * 128;
-        uint32_t r[64];
-        tmem_ld32(tm_s + col0, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
-        tmem_ld32(tm_s + col0 + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
+        if (!preloaded) {
+          checked(mbar_wait(&bars->s_full[sb], (g >> 1) & 1, abort_flag));
+          tc_fence_after();
+          const uint32_t tm_s = tmem + lane_addr + C::TM_S0 + sb * 128;
+          tmem_ld32(tm_s + col0, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
+          tmem_ld32(tm_s + col0 + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
+        }
         // the mask bits of a PARTIAL tile are computed while the load is in flight
         const bool part = (fl & part_bit) != 0;
         uint32_t mw[4] = {0xffffffffu, 0xffffffffu, 0xffffffffu, 0xffffffffu};
@@ -385,6 +401,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
           }
         }
         tmem_wait_ld();
+        regs_ready(*reinterpret_cast<uint32_t(*)[32]>(&r[0]));
+        regs_ready(*reinterpret_cast<uint32_t(*)[32]>(&r[32]));
         // S buffer sb may now take S_{g+2}
         warp_arrive(&bars->s_empty[sb]);
         float acc[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
@@ -422,6 +440,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
           checked(mbar_wait(&bars->pv_done[sb], ((g >> 1) - 1) & 1, abort_flag));
           tc_fence_after();
         }
+        // the next column's S is loaded into r as this column's P frees it
+        const bool next_in = j + 1 < n && (fl_next & in_bit);
+        const uint32_t sbn = (g + 1) & 1;
+        const uint32_t tm_sn = tmem + lane_addr + C::TM_S0 + sbn * 128;
         uint64_t acc2[2] = {0ull, 0ull};
 #pragma unroll
         for (int c = 0; c < 2; ++c) {
@@ -429,24 +451,36 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
           if (!(live & (1u << c))) {
 #pragma unroll
             for (int e = 0; e < 16; ++e) w[e] = 0u;
-            tmem_st16(tm_p + c * 16, w);
-            continue;
-          }
+          } else {
 #pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            const int k2 = 32 * c + 2 * e;
-            const uint64_t xs = f2_fma(f2_pack(__uint_as_float(r[k2]), __uint_as_float(r[k2 + 1])), sl2, negm);
-            float x0, x1;
-            f2_unpack(xs, x0, x1);
-            const uint64_t pe = f2_pack(ex2_approx(x0), ex2_approx(x1));
-            acc2[e & 1] = f2_add(acc2[e & 1], pe);
-            float q0, q1;
-            f2_unpack(pe, q0, q1);
-            w[e] = pack_bf16x2(q0, q1);
+            for (int e = 0; e < 16; ++e) {
+              const int k2 = 32 * c + 2 * e;
+              const uint64_t xs = f2_fma(f2_pack(__uint_as_float(r[k2]), __uint_as_float(r[k2 + 1])), sl2, negm);
+              uint64_t pe;
+              if (exp2_on_fma(e)) {
+                pe = exp2_fma_x2(xs);
+              } else {
+                float x0, x1;
+                f2_unpack(xs, x0, x1);
+                pe = f2_pack(ex2_approx(x0), ex2_approx(x1));
+              }
+              acc2[e & 1] = f2_add(acc2[e & 1], pe);
+              float q0, q1;
+              f2_unpack(pe, q0, q1);
+              w[e] = pack_bf16x2(q0, q1);
+            }
           }
           // P (bf16 pairs) of keys [col0 + 32 c, +32) -> P columns (col0 + 32 c) / 2
           tmem_st16(tm_p + c * 16, w);
+          if (next_in) {
+            if (c == 0) {
+              checked(mbar_wait(&bars->s_full[sbn], ((g + 1) >> 1) & 1, abort_flag));
+              tc_fence_after();
+            }
+            tmem_ld32(tm_sn + col0 + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(&r[32 * c]));
+          }
         }
+        preloaded = next_in;
         const uint64_t s01 = f2_add(acc2[0], acc2[1]);
         float s0, s1;
         f2_unpack(s01, s0, s1);
@@ -462,6 +496,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
             uint32_t ro[32];
             tmem_ld32(tm_o + c * 32, ro);
             tmem_wait_ld();
+            regs_ready(ro);
 #pragma unroll
             for (int e = 0; e < 32; ++e) ro[e] = __float_as_uint(__uint_as_float(ro[e]) * factor);
             tmem_st32(tm_o + c * 32, ro);

@@ -232,6 +232,20 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
       : "r"(taddr));
 }
 
+// Tie the destination registers of earlier tcgen05.ld to a point after
+// tcgen05.wait::ld: the loads complete asynchronously, so no use of these
+// registers may be scheduled before the wait.  Emits no instruction.
+__device__ __forceinline__ void regs_ready(uint32_t (&r)[32]) {
+  asm volatile(""
+               : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]),
+                 "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]),
+                 "+r"(r[14]), "+r"(r[15]), "+r"(r[16]), "+r"(r[17]), "+r"(r[18]), "+r"(r[19]),
+                 "+r"(r[20]), "+r"(r[21]), "+r"(r[22]), "+r"(r[23]), "+r"(r[24]), "+r"(r[25]),
+                 "+r"(r[26]), "+r"(r[27]), "+r"(r[28]), "+r"(r[29]), "+r"(r[30]), "+r"(r[31])
+               :
+               : "memory");
+}
+
 __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
   asm volatile(
       "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
@@ -451,6 +465,34 @@ __device__ __forceinline__ float max3f(float a, float b, float c) {
   float d;
   asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
   return d;
+}
+
+// 2^x for two lanes on the FMA and integer pipes instead of the MUFU: range
+// reduction x = j + f with j = round(x) (adding 1.5 * 2^23 leaves j in the low
+// mantissa bits) and f in [-1/2, 1/2], a cubic for 2^f, and j added to the
+// exponent field.  The cubic's coefficients are a least-squares fit in
+// relative error, reweighted towards equal ripple (Lawson's iteration), on
+// [-1/2, 1/2]; maximum relative error 8.4e-5, far below bf16's 2^-8 step
+// (tests/test_exp2_fma.py re-derives them).  Inputs are clamped at -125 so
+// the result stays a normal float (about 2.4e-38 for -inf).
+__device__ __forceinline__ uint64_t exp2_fma_x2(uint64_t x) {
+  float x0, x1;
+  f2_unpack(x, x0, x1);
+  const uint64_t xx = f2_pack(fmaxf(x0, -125.0f), fmaxf(x1, -125.0f));
+  const uint64_t kShift = f2_pack(12582912.0f, 12582912.0f);  // 1.5 * 2^23
+  const uint64_t t = f2_add(xx, kShift);
+  const uint64_t jf = f2_add(t, f2_pack(-12582912.0f, -12582912.0f));  // round(x) as a float
+  const uint64_t f = f2_fma(jf, f2_pack(-1.0f, -1.0f), xx);           // x - round(x)
+  uint64_t q = f2_fma(f2_pack(0.055212993174791336f, 0.055212993174791336f), f,
+                      f2_pack(0.24271413683891296f, 0.24271413683891296f));
+  q = f2_fma(q, f, f2_pack(0.6932621598243713f, 0.6932621598243713f));
+  q = f2_fma(q, f, f2_pack(0.999919593334198f, 0.999919593334198f));
+  float t0, t1, q0, q1;
+  f2_unpack(t, t0, t1);
+  f2_unpack(q, q0, q1);
+  const int j0 = __float_as_int(t0) - 0x4B400000;
+  const int j1 = __float_as_int(t1) - 0x4B400000;
+  return f2_pack(__int_as_float(__float_as_int(q0) + (j0 << 23)), __int_as_float(__float_as_int(q1) + (j1 << 23)));
 }
 
 // Named barrier over the first `nthreads` threads that reach barrier `id`
