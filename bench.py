@@ -515,16 +515,13 @@ def run_lora_layer(wl, csr, dev, stream, r):
 
 
 def fwd_kernel_name():
-    k = os.environ.get("RADIAL_FWD_KERNEL", "")
-    return {"single": "radial_fwd_kernel<128>", "cta2": "radial_fwd_cta2_kernel<128>"}.get(
-        k, "radial_fwd_pair_kernel<128>")
+    return "radial_fwd_pair_kernel<128>"
 
 
 def kernel_sha():
     import hashlib
     h = hashlib.sha1()
-    for f in ("attn_fwd.cuh", "attn_fwd_pair.cuh", "attn_fwd_cta2.cuh", "sm100_primitives.cuh", "mask_build.cuh",
-              "radial_lib.cu"):
+    for f in ("attn_fwd.cuh", "attn_fwd_pair.cuh", "sm100_primitives.cuh", "mask_build.cuh", "radial_lib.cu"):
         with open(os.path.join(ROOT, "block_sparse_attention_csr_b200", "csrc", f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:12]

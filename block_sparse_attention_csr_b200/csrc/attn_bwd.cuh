@@ -624,7 +624,7 @@ __global__ void __launch_bounds__(384, 1)
         if (partial) {
           mw[0] = mw[1] = mw[2] = mw[3] = 0u;
           if (valid) {
-            FwdParams mp{};
+            RowMaskGeom mp{};
             mp.f = p.f;
             mp.s = p.s;
             mp.n = p.n;

@@ -303,7 +303,7 @@ __global__ void __launch_bounds__(384, 1)
       return *x_peer;
     };
     constexpr float kRescaleThreshold = 8.0f;
-    FwdParams mp{};
+    RowMaskGeom mp{};
     mp.f = p.f;
     mp.s = p.s;
     mp.n = p.n;

@@ -22,7 +22,6 @@
 #include "attn_bwd.cuh"
 #include "attn_fwd.cuh"
 #include "attn_fwd_pair.cuh"
-#include "attn_fwd_cta2.cuh"
 #include "mask_build.cuh"
 #include "sm100_primitives.cuh"
 
@@ -508,58 +507,8 @@ float softmax_scale(const radial_desc* d) {
   return d->scale > 0.f ? d->scale : 1.0f / std::sqrt(static_cast<float>(d->head_dim));
 }
 
-// Work-item order inside a head.  Default: longest row (column) first, which
-// measured best (it balances the tail of each launch).
-// RADIAL_SCHEDULE=natural: ascending tile position (the CTAs running at the
-// same time then share the K / V of a band of nearby frames).
-bool schedule_lpt() {
-  static const bool lpt = [] {
-    const char* e = std::getenv("RADIAL_SCHEDULE");
-    return !(e && std::strcmp(e, "natural") == 0);
-  }();
-  return lpt;
-}
-
-// Forward kernel choice: 0 two tiles per CTA (default), 1 one tile per CTA,
-// 2 one tile per CTA with the MMA shared by a CTA pair (RADIAL_FWD_KERNEL =
-// pair | single | cta2).
-int fwd_kernel_choice() {
-  static const int k = [] {
-    const char* e = std::getenv("RADIAL_FWD_KERNEL");
-    if (e && std::strcmp(e, "single") == 0) return 1;
-    if (e && std::strcmp(e, "cta2") == 0) return 2;
-    return 0;
-  }();
-  return k;
-}
-
-// Number of 2-CTA clusters of the CTA-pair forward that fit on the device at
-// once (looked up once per device).
-int pair_clusters(int smem) {
-  static int cached[64] = {};
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return sm_count() / 2;
-  if (cached[dev] > 0) return cached[dev];
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(2 * (sm_count() / 2), 1, 1);
-  cfg.blockDim = dim3(384, 1, 1);
-  cfg.dynamicSmemBytes = static_cast<size_t>(smem);
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = 2;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  int n = 0;
-  if (cudaOccupancyMaxActiveClusters(&n, radial_fwd_cta2_kernel<128>, &cfg) != cudaSuccess || n <= 0) {
-    cudaGetLastError();
-    n = sm_count() / 2;
-  }
-  cached[dev] = n;
-  return n;
-}
-
+// Work items run head-major and, inside a head, longest row (column) first:
+// the order arrays built with the mask.  It balances the tail of each launch.
 template <int D>
 radial_status launch_fwd_pair(const radial_csr* c, const radial_desc* d, const void* q, const void* k,
                               const void* v, void* o, float* lse, cudaStream_t st) {
@@ -572,7 +521,7 @@ radial_status launch_fwd_pair(const radial_csr* c, const radial_desc* d, const v
   p.pair_ptr = c->pairs.ptr;
   p.pair_col = c->pairs.col;
   p.pair_flag = c->pairs.flag;
-  p.pair_order = schedule_lpt() ? c->pairs.order : nullptr;
+  p.pair_order = c->pairs.order;
   p.hd = c->hd;
   p.cd = c->cd;
   p.np = c->pairs.np;
@@ -593,79 +542,6 @@ radial_status launch_fwd_pair(const radial_csr* c, const radial_desc* d, const v
   const int grid = p.items < sm_count() ? p.items : sm_count();
   RADIAL_CUDA(cudaFuncSetAttribute(radial_fwd_pair_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
   radial_fwd_pair_kernel<D><<<grid, 384, smem, st>>>(mq, mk, mv, p);
-  RADIAL_LAUNCHED();
-  return RADIAL_OK;
-}
-
-radial_status launch_fwd_cta2(const radial_csr* c, const radial_desc* d, const void* q, const void* k,
-                              const void* v, void* o, float* lse, cudaStream_t st) {
-  CUtensorMap mq, mk, mv;
-  radial_status rs;
-  if ((rs = make_bhnd_map(&mq, q, *d)) != RADIAL_OK) return rs;
-  if ((rs = make_bhnd_map(&mk, k, *d, 64)) != RADIAL_OK) return rs;   // a CTA loads 64 keys of a tile
-  if ((rs = make_bhnd_map(&mv, v, *d)) != RADIAL_OK) return rs;       // and 64 columns of its values
-  FwdPairParams p;
-  p.pair_ptr = c->pairs.ptr;
-  p.pair_col = c->pairs.col;
-  p.pair_flag = c->pairs.flag;
-  p.pair_order = schedule_lpt() ? c->pairs.order : nullptr;
-  p.hd = c->hd;
-  p.cd = c->cd;
-  p.np = c->pairs.np;
-  p.nt = c->plan.nb;
-  p.f = c->f;
-  p.s = c->s;
-  p.n = c->n;
-  p.sink = c->sink;
-  p.heads = d->heads;
-  p.items = d->batch * d->heads * c->pairs.np;
-  p.o_sb = d->stride_b;
-  p.o_sh = d->stride_h;
-  p.o_sn = d->stride_n;
-  p.o = reinterpret_cast<__nv_bfloat16*>(o);
-  p.lse = lse;
-  p.scale_log2 = softmax_scale(d) * 1.4426950408889634f;
-  const int smem = FwdCta2Cfg<128>::SMEM_BYTES;
-  RADIAL_CUDA(cudaFuncSetAttribute(radial_fwd_cta2_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
-  const int clusters = pair_clusters(smem);
-  const int grid = 2 * (p.items < clusters ? p.items : clusters);
-  radial_fwd_cta2_kernel<128><<<grid, 384, smem, st>>>(mq, mk, mv, p);
-  RADIAL_LAUNCHED();
-  return RADIAL_OK;
-}
-
-template <int D>
-radial_status launch_fwd(const radial_csr* c, const radial_desc* d, const void* q, const void* k,
-                         const void* v, void* o, float* lse, cudaStream_t st) {
-  CUtensorMap mq, mk, mv;
-  radial_status rs;
-  if ((rs = make_bhnd_map(&mq, q, *d)) != RADIAL_OK) return rs;
-  if ((rs = make_bhnd_map(&mk, k, *d)) != RADIAL_OK) return rs;
-  if ((rs = make_bhnd_map(&mv, v, *d)) != RADIAL_OK) return rs;
-  FwdParams p;
-  p.row_ptr = c->plan.row_ptr;
-  p.col_idx = c->plan.col_idx;
-  p.kind = c->plan.kind;
-  p.order = schedule_lpt() ? c->plan.row_order : nullptr;
-  p.hd = c->hd;
-  p.cd = c->cd;
-  p.nt = c->plan.nb;
-  p.f = c->f;
-  p.s = c->s;
-  p.n = c->n;
-  p.sink = c->sink;
-  p.heads = d->heads;
-  p.items = d->batch * d->heads * c->plan.nb;
-  p.o_sb = d->stride_b;
-  p.o_sh = d->stride_h;
-  p.o_sn = d->stride_n;
-  p.o = reinterpret_cast<__nv_bfloat16*>(o);
-  p.lse = lse;
-  p.scale_log2 = softmax_scale(d) * 1.4426950408889634f;
-  const int smem = FwdCfg<D>::SMEM_BYTES;
-  const int grid = p.items < sm_count() ? p.items : sm_count();
-  RADIAL_CUDA(cudaFuncSetAttribute(radial_fwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
-  radial_fwd_kernel<D><<<grid, 384, smem, st>>>(mq, mk, mv, p);
   RADIAL_LAUNCHED();
   return RADIAL_OK;
 }
@@ -699,11 +575,11 @@ radial_status launch_bwd(const radial_csr* c, const radial_desc* d, const void* 
   p.row_ptr = c->plan.row_ptr;
   p.col_idx = c->plan.col_idx;
   p.kind = c->plan.kind;
-  p.row_order = schedule_lpt() ? c->plan.row_order : nullptr;
+  p.row_order = c->plan.row_order;
   p.col_ptr = c->plan.col_ptr;
   p.row_idx = c->plan.row_idx;
   p.kind_t = c->plan.kind_t;
-  p.col_order = schedule_lpt() ? c->plan.col_order : nullptr;
+  p.col_order = c->plan.col_order;
   p.hd = c->hd;
   p.cd = c->cd;
   p.nt = c->plan.nb;
@@ -743,14 +619,8 @@ radial_status radial_attn_fwd(const radial_csr* c, const radial_desc* d, const v
   if (!q || !k || !v || !o || !lse) return fail(RADIAL_EINVAL, "NULL tensor pointer");
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
     return fail(RADIAL_EINVAL, "tensor pointers must be 16-byte aligned");
-  const int choice = fwd_kernel_choice();
-  if (choice == 2 && d->head_dim == 128) return launch_fwd_cta2(c, d, q, k, v, o, lse, as_stream(stream));
-  if (choice != 1) {
-    if (d->head_dim == 128) return launch_fwd_pair<128>(c, d, q, k, v, o, lse, as_stream(stream));
-    return launch_fwd_pair<64>(c, d, q, k, v, o, lse, as_stream(stream));
-  }
-  if (d->head_dim == 128) return launch_fwd<128>(c, d, q, k, v, o, lse, as_stream(stream));
-  return launch_fwd<64>(c, d, q, k, v, o, lse, as_stream(stream));
+  if (d->head_dim == 128) return launch_fwd_pair<128>(c, d, q, k, v, o, lse, as_stream(stream));
+  return launch_fwd_pair<64>(c, d, q, k, v, o, lse, as_stream(stream));
 }
 
 size_t radial_attn_bwd_workspace_size(const radial_desc* d) {

@@ -232,20 +232,6 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
       : "r"(taddr));
 }
 
-// Tie the destination registers of earlier tcgen05.ld to a point after
-// tcgen05.wait::ld: the loads complete asynchronously, so no use of these
-// registers may be scheduled before the wait.  Emits no instruction.
-__device__ __forceinline__ void regs_ready(uint32_t (&r)[32]) {
-  asm volatile(""
-               : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]),
-                 "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]),
-                 "+r"(r[14]), "+r"(r[15]), "+r"(r[16]), "+r"(r[17]), "+r"(r[18]), "+r"(r[19]),
-                 "+r"(r[20]), "+r"(r[21]), "+r"(r[22]), "+r"(r[23]), "+r"(r[24]), "+r"(r[25]),
-                 "+r"(r[26]), "+r"(r[27]), "+r"(r[28]), "+r"(r[29]), "+r"(r[30]), "+r"(r[31])
-               :
-               : "memory");
-}
-
 __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
   asm volatile(
       "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
@@ -266,140 +252,6 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t* r) {
       "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
       "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
       "r"(r[15])
-      : "memory");
-}
-
-// ---------------------------------------------------------------------------
-// CTA pairs (cta_group::2): the two CTAs of a 2-CTA cluster share one MMA.
-// The even CTA (rank 0) issues every tcgen05.mma for both; A and the
-// accumulator are split by rows (128 per CTA), B by its N dimension (N/2
-// rows of B in each CTA's shared memory, at the same offset).
-// ---------------------------------------------------------------------------
-__device__ __forceinline__ uint32_t cluster_ctarank() {
-  uint32_t r;
-  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
-  return r;
-}
-__device__ __forceinline__ uint32_t cluster_id_x() {
-  uint32_t r;
-  asm volatile("mov.u32 %0, %%clusterid.x;" : "=r"(r));
-  return r;
-}
-__device__ __forceinline__ uint32_t cluster_count_x() {
-  uint32_t r;
-  asm volatile("mov.u32 %0, %%nclusterid.x;" : "=r"(r));
-  return r;
-}
-
-// Every thread of every CTA of the cluster (aligned: all threads execute it).
-__device__ __forceinline__ void cluster_sync_all() {
-  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
-}
-
-// The shared::cluster address of the object at the same offset in CTA `rank`.
-__device__ __forceinline__ uint32_t mapa_shared(uint32_t local_addr, uint32_t rank) {
-  uint32_t r;
-  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(local_addr), "r"(rank));
-  return r;
-}
-
-// Arrive on an mbarrier named by a shared::cluster address, possibly in the
-// other CTA of the pair.  The default (release, CTA scope) semantics are
-// enough: what a remote arrival publishes is TMEM state, ordered by the
-// tcgen05 fences around it, not ordinary memory; a cluster-scope release
-// would fence every arrival.
-__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
-  asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
-}
-
-__device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t* bar, uint32_t parity) {
-  return mbar_try_wait(bar, parity);
-}
-
-// Bounded wait (as mbar_wait) for barriers that the other CTA of the pair
-// arrives on.
-__device__ __forceinline__ bool mbar_wait_cl(uint64_t* bar, uint32_t parity, volatile int* abort) {
-  if (mbar_try_wait_cluster(bar, parity)) return true;
-  const uint64_t t0 = globaltimer_ns();
-  uint32_t spins = 0;
-  while (true) {
-    if (*abort) return false;
-    if (mbar_try_wait_cluster(bar, parity)) return true;
-    if ((++spins & 63u) == 0u && globaltimer_ns() - t0 > kWaitLimitNs) {
-      *abort = 1;
-      atomicExch(&g_device_error, kErrWaitTimeout);
-      return false;
-    }
-  }
-}
-
-__device__ __forceinline__ bool mbar_wait_drain_cl(uint64_t* bar, uint32_t parity) {
-  if (mbar_try_wait_cluster(bar, parity)) return true;
-  const uint64_t t0 = globaltimer_ns();
-  uint32_t spins = 0;
-  while (true) {
-    if (mbar_try_wait_cluster(bar, parity)) return true;
-    if ((++spins & 63u) == 0u && globaltimer_ns() - t0 > kWaitLimitNs) {
-      atomicExch(&g_device_error, kErrWaitTimeout);
-      return false;
-    }
-  }
-}
-
-// Tiled TMA load into this CTA's shared memory whose completion is counted
-// on an mbarrier of either CTA of the pair (bar_cluster: a shared::cluster
-// address, normally the even CTA's barrier).  No multicast.
-__device__ __forceinline__ void tma_load_4d_pair(void* smem_dst, const CUtensorMap* map, uint32_t bar_cluster,
-                                                 int c0, int c1, int c2, int c3) {
-  asm volatile(
-      "cp.async.bulk.tensor.4d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%3, %4, %5, %6}], [%2];" ::"r"(smem_u32(smem_dst)),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar_cluster), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
-      : "memory");
-}
-
-// TMEM allocation for a CTA pair: one warp of EACH CTA (same warp index)
-// executes these; both CTAs get the same columns.
-__device__ __forceinline__ void tmem_alloc_pair(uint32_t* smem_result, uint32_t ncols) {
-  asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(smem_result)),
-               "r"(ncols)
-               : "memory");
-}
-__device__ __forceinline__ void tmem_relinquish_pair() {
-  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
-}
-__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
-  asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
-}
-
-// M = 256 MMAs over the pair (issued by the even CTA only), kind::f16.
-__device__ __forceinline__ void mma_ss_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
-                                            uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-__device__ __forceinline__ void mma_ts_pair(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
-                                            uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::2.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-
-// Arrive once on the mbarrier at this offset in BOTH CTAs of the pair when
-// every tcgen05 op issued so far by this thread has completed.
-__device__ __forceinline__ void mma_commit_pair(uint64_t* bar) {
-  asm volatile(
-      "{\n\t.reg .b16 m;\n\t"
-      "mov.b16 m, 3;\n\t"
-      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], m;\n\t}" ::"r"(
-          smem_u32(bar))
       : "memory");
 }
 
@@ -465,34 +317,6 @@ __device__ __forceinline__ float max3f(float a, float b, float c) {
   float d;
   asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
   return d;
-}
-
-// 2^x for two lanes on the FMA and integer pipes instead of the MUFU: range
-// reduction x = j + f with j = round(x) (adding 1.5 * 2^23 leaves j in the low
-// mantissa bits) and f in [-1/2, 1/2], a cubic for 2^f, and j added to the
-// exponent field.  The cubic's coefficients are a least-squares fit in
-// relative error, reweighted towards equal ripple (Lawson's iteration), on
-// [-1/2, 1/2]; maximum relative error 8.4e-5, far below bf16's 2^-8 step
-// (tests/test_exp2_fma.py re-derives them).  Inputs are clamped at -125 so
-// the result stays a normal float (about 2.4e-38 for -inf).
-__device__ __forceinline__ uint64_t exp2_fma_x2(uint64_t x) {
-  float x0, x1;
-  f2_unpack(x, x0, x1);
-  const uint64_t xx = f2_pack(fmaxf(x0, -125.0f), fmaxf(x1, -125.0f));
-  const uint64_t kShift = f2_pack(12582912.0f, 12582912.0f);  // 1.5 * 2^23
-  const uint64_t t = f2_add(xx, kShift);
-  const uint64_t jf = f2_add(t, f2_pack(-12582912.0f, -12582912.0f));  // round(x) as a float
-  const uint64_t f = f2_fma(jf, f2_pack(-1.0f, -1.0f), xx);           // x - round(x)
-  uint64_t q = f2_fma(f2_pack(0.055212993174791336f, 0.055212993174791336f), f,
-                      f2_pack(0.24271413683891296f, 0.24271413683891296f));
-  q = f2_fma(q, f, f2_pack(0.6932621598243713f, 0.6932621598243713f));
-  q = f2_fma(q, f, f2_pack(0.999919593334198f, 0.999919593334198f));
-  float t0, t1, q0, q1;
-  f2_unpack(t, t0, t1);
-  f2_unpack(q, q0, q1);
-  const int j0 = __float_as_int(t0) - 0x4B400000;
-  const int j1 = __float_as_int(t1) - 0x4B400000;
-  return f2_pack(__int_as_float(__float_as_int(q0) + (j0 << 23)), __int_as_float(__float_as_int(q1) + (j1 << 23)));
 }
 
 // Named barrier over the first `nthreads` threads that reach barrier `id`

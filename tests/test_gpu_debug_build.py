@@ -17,10 +17,9 @@ pytestmark = pytest.mark.gpu
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 
-@pytest.mark.parametrize("kernel", ["pair", "cta2"])
-def test_parity_through_the_debug_build(kernel):
+def test_parity_through_the_debug_build():
     build_mod.build()
-    env = dict(os.environ, RADIAL_LIBRARY=build_mod.OUT_DEBUG, RADIAL_FWD_KERNEL=kernel)
+    env = dict(os.environ, RADIAL_LIBRARY=build_mod.OUT_DEBUG)
     r = subprocess.run([sys.executable, "-m", "pytest", "-q", "-p", "no:cacheprovider", "-m", "gpu",
                         os.path.join(ROOT, "tests", "test_gpu_fwd.py"), os.path.join(ROOT, "tests", "test_gpu_bwd.py"),
                         "-k", "test_small_all_rows or test_small_all_gradients or test_tiny_config"],

@@ -166,35 +166,3 @@ def test_many_work_items_all_rows():
     res = oracle_pool.run("fwd_rows", tasks)
     _check(o[0].float().cpu().numpy().reshape(-1, 128), lse[0].cpu().numpy().reshape(-1),
            np.concatenate([a for a, _ in res]), np.concatenate([b for _, b in res]), "many items")
-
-
-def test_cta_pair_kernel_all_rows():
-    """The forward with the MMA shared by a CTA pair (tcgen05 cta_group::2,
-    head_dim 128; head_dim 64 cases run the default kernel), selected per
-    process by RADIAL_FWD_KERNEL=cta2: the all-row parity cases above, in a
-    child process with that variable set."""
-    import subprocess
-    import sys
-    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
-    env = dict(os.environ, RADIAL_FWD_KERNEL="cta2")
-    r = subprocess.run([sys.executable, "-m", "pytest", os.path.join(root, "tests", "test_gpu_fwd.py"), "-q",
-                        "-p", "no:cacheprovider", "-m", "gpu",
-                        "-k", "test_tiny_config_all_rows or test_small_all_rows or test_strided_layout or "
-                              "test_dense_mask or test_repeated_calls or test_many_work_items"],
-                       cwd=root, env=env, capture_output=True, text=True, timeout=1200)
-    assert r.returncode == 0, r.stdout[-3000:] + r.stderr[-2000:]
-
-
-def test_one_tile_kernel_all_rows():
-    """The alternate forward (one query tile per CTA, double-buffered S),
-    selected per process by RADIAL_FWD_KERNEL=single: the all-row parity
-    cases above, run in a child process with that variable set."""
-    import subprocess
-    import sys
-    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
-    env = dict(os.environ, RADIAL_FWD_KERNEL="single")
-    r = subprocess.run([sys.executable, "-m", "pytest", os.path.join(root, "tests", "test_gpu_fwd.py"), "-q",
-                        "-p", "no:cacheprovider", "-m", "gpu",
-                        "-k", "test_tiny_config_all_rows or test_small_all_rows or test_strided_layout"],
-                       cwd=root, env=env, capture_output=True, text=True, timeout=1200)
-    assert r.returncode == 0, r.stdout[-3000:] + r.stderr[-2000:]
