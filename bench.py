@@ -481,7 +481,8 @@ def run_sweep(args, dev, stream, peak):
 def run_lora_layer(wl, csr, dev, stream, r):
     """One LoRA-adapted attention layer step (forward + backward: dx and the
     adapter gradients) at the workload's shape, hidden size heads*head_dim,
-    adapter rank r: projections in cuBLAS, attention in the library."""
+    adapter rank r: projections on the library's tensor-core GEMM, attention
+    in its block-sparse kernels."""
     import numpy as np
     import torch
     from block_sparse_attention_csr_b200 import inputs as I
@@ -511,7 +512,7 @@ def run_lora_layer(wl, csr, dev, stream, r):
     del t, layer
     torch.cuda.empty_cache()
     return {"rank": r, "hidden": C, "ms_per_step": ms, "projection_gemm_tflop": proj_flops / 1e12,
-            "path": "4 LoRA projections (cuBLAS GEMMs) + radial_attn_fwd/bwd (this library), forward + backward"}
+            "path": "4 LoRA projections (radial_lora_fwd/bwd) + radial_attn_fwd/bwd, all in this library, forward + backward"}
 
 
 def fwd_kernel_name():

@@ -20,6 +20,8 @@ from ._binding import (  # noqa: F401
     radial_csr_info,
     radial_device_status,
     radial_launch_count,
+    radial_lora_bwd,
+    radial_lora_fwd,
     radial_mask_build,
     radial_mask_build_dense,
     radial_params_default,

@@ -30,7 +30,7 @@ EXPORTED = (
     "radial_csr_copy_to_host", "radial_csr_free", "radial_attn_fwd",
     "radial_attn_bwd_workspace_size", "radial_attn_bwd", "radial_device_status",
     "radial_status_str", "radial_last_error", "radial_launch_count", "radial_selftest_bounded_wait",
-    "radial_attn_bwd_noalloc",
+    "radial_attn_bwd_noalloc", "radial_lora_fwd", "radial_lora_bwd_workspace_size", "radial_lora_bwd",
 )
 
 
@@ -97,6 +97,13 @@ def load(path=None):
         L.radial_attn_bwd.restype = ctypes.c_int
         L.radial_attn_bwd_noalloc.argtypes = [vp, ctypes.POINTER(radial_desc)] + [vp] * 10
         L.radial_attn_bwd_noalloc.restype = ctypes.c_int
+        L.radial_lora_fwd.argtypes = [i64, i32, i32, i32, ctypes.c_float, vp, i64, vp, vp, vp, vp, i64, vp, vp]
+        L.radial_lora_fwd.restype = ctypes.c_int
+        L.radial_lora_bwd_workspace_size.argtypes = [i64, i32, i32, i32]
+        L.radial_lora_bwd_workspace_size.restype = sz
+        L.radial_lora_bwd.argtypes = [i64, i32, i32, i32, ctypes.c_float, vp, i64, vp, i64, vp, vp, vp, vp, vp, i64,
+                                      i32, vp, vp, vp, sz, vp]
+        L.radial_lora_bwd.restype = ctypes.c_int
         L.radial_device_status.argtypes = [vp]
         L.radial_device_status.restype = ctypes.c_int
         L.radial_status_str.argtypes = [ctypes.c_int]
@@ -278,6 +285,54 @@ def radial_attn_bwd_noalloc(csr, do, q, k, v, o, lse, dq=None, dk=None, dv=None,
                                           _ptr(o), _ptr(lse), _ptr(dq), _ptr(dk), _ptr(dv), _stream(stream)),
            "radial_attn_bwd_noalloc")
     return dq, dk, dv
+
+
+def _rows(t, what):
+    """(rows, cols, row stride) of a 2-D bf16 CUDA tensor with unit column stride."""
+    import torch
+    if t.dim() != 2 or t.stride(1) != 1 or t.dtype != torch.bfloat16 or not t.is_cuda:
+        raise ValueError(f"{what}: expected a 2-D CUDA bf16 tensor with contiguous rows")
+    return t.shape[0], t.shape[1], t.stride(0)
+
+
+def radial_lora_fwd(x, W, A, B, scale, y=None, u=None, stream=None):
+    """y = x W^T + s (x A^T) B^T on the library's tensor-core GEMMs.
+    x [n, c_in], W [c_out, c_in], A [r, c_in], B [c_out, r].  Returns (y, u)
+    with u = s x A^T, which radial_lora_bwd takes back."""
+    import torch
+    n, c_in, ldx = _rows(x, "x")
+    c_out, r = W.shape[0], A.shape[0]
+    for t, shape, nm in ((W, (c_out, c_in), "W"), (A, (r, c_in), "A"), (B, (c_out, r), "B")):
+        if tuple(t.shape) != shape or not t.is_contiguous():
+            raise ValueError(f"{nm}: expected a contiguous {shape} tensor")
+    y = torch.empty(n, c_out, dtype=torch.bfloat16, device=x.device) if y is None else y
+    u = torch.empty(n, r, dtype=torch.bfloat16, device=x.device) if u is None else u
+    _, _, ldy = _rows(y, "y")
+    _check(load().radial_lora_fwd(n, c_in, c_out, r, float(scale), _ptr(x), ldx, _ptr(W), _ptr(A), _ptr(B),
+                                  _ptr(y), ldy, _ptr(u), _stream(stream)), "radial_lora_fwd")
+    return y, u
+
+
+def radial_lora_bwd(dy, x, W, A, B, u, scale, dx=None, accumulate_dx=False, dA=None, dB=None, workspace=None,
+                    stream=None):
+    """(dx, dA, dB) of radial_lora_fwd for upstream dy [n, c_out]; with
+    accumulate_dx the result is added to the given dx."""
+    import torch
+    n, c_out, lddy = _rows(dy, "dy")
+    _, c_in, ldx = _rows(x, "x")
+    r = A.shape[0]
+    dx = torch.empty(n, c_in, dtype=torch.bfloat16, device=x.device) if dx is None else dx
+    dA = torch.empty(r, c_in, dtype=torch.bfloat16, device=x.device) if dA is None else dA
+    dB = torch.empty(c_out, r, dtype=torch.bfloat16, device=x.device) if dB is None else dB
+    _, _, lddx = _rows(dx, "dx")
+    need = int(load().radial_lora_bwd_workspace_size(n, c_in, c_out, r))
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=x.device)
+    _check(load().radial_lora_bwd(n, c_in, c_out, r, float(scale), _ptr(dy), lddy, _ptr(x), ldx, _ptr(W), _ptr(A),
+                                  _ptr(B), _ptr(u), _ptr(dx), lddx, 1 if accumulate_dx else 0, _ptr(dA), _ptr(dB),
+                                  _ptr(workspace), ctypes.c_size_t(workspace.numel() * workspace.element_size()),
+                                  _stream(stream)), "radial_lora_bwd")
+    return dx, dA, dB
 
 
 def radial_device_status(stream=None):

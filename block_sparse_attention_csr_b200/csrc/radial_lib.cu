@@ -8,6 +8,7 @@
 #include <cuda_runtime.h>
 #include <nvtx3/nvToolsExt.h>
 
+#include <algorithm>
 #include <atomic>
 #include <cmath>
 #include <cstdarg>
@@ -22,6 +23,7 @@
 #include "attn_bwd.cuh"
 #include "attn_fwd.cuh"
 #include "attn_fwd_pair.cuh"
+#include "gemm.cuh"
 #include "mask_build.cuh"
 #include "sm100_primitives.cuh"
 
@@ -761,5 +763,219 @@ const char* radial_status_str(radial_status s) {
 const char* radial_last_error(void) { return t_last_error.c_str(); }
 
 int64_t radial_launch_count(void) { return g_launches.load(); }
+
+}  // extern "C"
+
+// ---------------------------------------------------------------------------
+// LoRA-adapted projections (the fine-tuning layer step around the attention)
+// ---------------------------------------------------------------------------
+namespace {
+
+// 2D map over a bf16 row-major [rows, cols] matrix with row stride ld
+// (elements): 64-column x 128-row boxes, 128-byte swizzle; outside reads 0.
+radial_status make_rowmajor_map(CUtensorMap* map, const void* base, int64_t rows, int64_t cols, int64_t ld) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return fail(RADIAL_ECUDA, "cuTensorMapEncodeTiled unavailable");
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld) * 2};
+  cuuint32_t box[2] = {64, 128};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(RADIAL_ECUDA, "cuTensorMapEncodeTiled (gemm operand) failed (%d)", static_cast<int>(r));
+  return RADIAL_OK;
+}
+
+// One operand pair of a GEMM segment: A [M, K] and B [N, K], both K-major.
+struct GemmSeg {
+  const void* a;
+  int64_t lda;
+  const void* b;
+  int64_t ldb;
+  int64_t k;  // 0: no segment
+};
+
+// C[M, N] = alpha (A0 B0^T + A1 B1^T) + beta C (bf16 c) or acc += ... (fp32,
+// split over K into up to `max_splits` slices).  Encodes every map first.
+radial_status launch_gemm(int64_t M, int64_t N, const GemmSeg& s0, const GemmSeg& s1, float alpha, float beta,
+                          void* c, float* acc, int64_t ldc, int max_splits, cudaStream_t st) {
+  CUtensorMap a0, b0, a1, b1;
+  radial_status rs;
+  if ((rs = make_rowmajor_map(&a0, s0.a, M, s0.k, s0.lda)) != RADIAL_OK) return rs;
+  if ((rs = make_rowmajor_map(&b0, s0.b, N, s0.k, s0.ldb)) != RADIAL_OK) return rs;
+  if (s1.k > 0) {
+    if ((rs = make_rowmajor_map(&a1, s1.a, M, s1.k, s1.lda)) != RADIAL_OK) return rs;
+    if ((rs = make_rowmajor_map(&b1, s1.b, N, s1.k, s1.ldb)) != RADIAL_OK) return rs;
+  } else {
+    a1 = a0;
+    b1 = b0;
+  }
+  GemmParams p;
+  p.M = static_cast<int32_t>(M);
+  p.N = static_cast<int32_t>(N);
+  p.kb0 = static_cast<int32_t>((s0.k + 63) / 64);
+  p.kb_total = p.kb0 + static_cast<int32_t>((s1.k + 63) / 64);
+  p.tiles_m = static_cast<int32_t>((M + 127) / 128);
+  p.tiles_n = static_cast<int32_t>((N + 127) / 128);
+  const int tiles = p.tiles_m * p.tiles_n;
+  int splits = 1;
+  if (acc) {  // split K until the grid fills the device
+    splits = std::max(1, std::min({max_splits, p.kb_total, (sm_count() + tiles - 1) / tiles}));
+  }
+  p.kb_per_split = (p.kb_total + splits - 1) / splits;
+  p.splits = (p.kb_total + p.kb_per_split - 1) / p.kb_per_split;  // every slice non-empty
+  p.items = tiles * p.splits;
+  p.alpha = alpha;
+  p.beta = beta;
+  p.c = reinterpret_cast<__nv_bfloat16*>(c);
+  p.acc = acc;
+  p.ldc = ldc;
+  RADIAL_CUDA(cudaFuncSetAttribute(radial_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                   GemmCfg::SMEM_BYTES));
+  const int grid = p.items < sm_count() ? p.items : sm_count();
+  radial_gemm_kernel<<<grid, 256, GemmCfg::SMEM_BYTES, st>>>(a0, b0, a1, b1, p);
+  RADIAL_LAUNCHED();
+  return RADIAL_OK;
+}
+
+radial_status launch_transpose(const void* in, int64_t ld_in, int64_t R, int64_t Cc, void* out, int64_t ld_out,
+                               cudaStream_t st) {
+  dim3 grid(static_cast<unsigned>((Cc + 31) / 32), static_cast<unsigned>((R + 31) / 32));
+  transpose_bf16_kernel<<<grid, dim3(32, 8), 0, st>>>(reinterpret_cast<const __nv_bfloat16*>(in), ld_in,
+                                                      static_cast<int>(R), static_cast<int>(Cc),
+                                                      reinterpret_cast<__nv_bfloat16*>(out), ld_out);
+  RADIAL_LAUNCHED();
+  return RADIAL_OK;
+}
+
+int64_t pad8(int64_t x) { return (x + 7) & ~int64_t(7); }
+size_t pad256(size_t x) { return (x + 255) & ~size_t(255); }
+
+// Workspace of radial_lora_bwd, carved in this order.
+struct LoraWs {
+  size_t wt, bt, at, v, vt, xt, dyt, ut, dA, dB, total;
+};
+LoraWs lora_ws(int64_t n, int64_t ci, int64_t co, int64_t r) {
+  const int64_t ln = pad8(n);
+  LoraWs w;
+  size_t o = 0;
+  w.wt = o; o += pad256(2 * ci * co);
+  w.bt = o; o += pad256(2 * r * co);
+  w.at = o; o += pad256(2 * ci * r);
+  w.v = o; o += pad256(2 * n * r);
+  w.vt = o; o += pad256(2 * r * ln);
+  w.xt = o; o += pad256(2 * ci * ln);
+  w.dyt = o; o += pad256(2 * co * ln);
+  w.ut = o; o += pad256(2 * r * ln);
+  w.dA = o; o += pad256(4 * r * ci);
+  w.dB = o; o += pad256(4 * co * r);
+  w.total = o;
+  return w;
+}
+
+radial_status check_lora(int64_t n, int32_t ci, int32_t co, int32_t r, int64_t ld1, int64_t ld2) {
+  if (n < 1 || ci < 1 || co < 1 || r < 1) return fail(RADIAL_EINVAL, "sizes must be >= 1");
+  if (n > 0x7fffffffLL) return fail(RADIAL_EUNSUPPORTED, "n_tokens beyond 2^31 - 1");
+  if (ci % 8 || co % 8 || r % 8) return fail(RADIAL_EINVAL, "c_in, c_out and rank must be multiples of 8");
+  if (ld1 % 8 || ld2 % 8) return fail(RADIAL_EINVAL, "row strides must be multiples of 8 elements");
+  return RADIAL_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+radial_status radial_lora_fwd(int64_t n, int32_t c_in, int32_t c_out, int32_t rank, float scale, const void* x,
+                              int64_t ldx, const void* W, const void* A, const void* B, void* y, int64_t ldy,
+                              void* u, void* stream) {
+  NvtxRange nvtx_range("radial_lora_fwd");
+  radial_status rs = check_lora(n, c_in, c_out, rank, ldx, ldy);
+  if (rs != RADIAL_OK) return rs;
+  if (!x || !W || !A || !B || !y || !u) return fail(RADIAL_EINVAL, "NULL pointer");
+  if (!aligned16(x) || !aligned16(W) || !aligned16(A) || !aligned16(B) || !aligned16(y) || !aligned16(u))
+    return fail(RADIAL_EINVAL, "pointers must be 16-byte aligned");
+  if (ldx < c_in || ldy < c_out) return fail(RADIAL_EINVAL, "row strides must cover the rows");
+  cudaStream_t st = as_stream(stream);
+  // u = s x A^T  [n, r]
+  GemmSeg none{nullptr, 0, nullptr, 0, 0};
+  if ((rs = launch_gemm(n, rank, GemmSeg{x, ldx, A, c_in, c_in}, none, scale, 0.f, u, nullptr, rank, 1, st)) !=
+      RADIAL_OK)
+    return rs;
+  // y = x W^T + u B^T  [n, c_out]
+  return launch_gemm(n, c_out, GemmSeg{x, ldx, W, c_in, c_in}, GemmSeg{u, rank, B, rank, rank}, 1.f, 0.f, y,
+                     nullptr, ldy, 1, st);
+}
+
+size_t radial_lora_bwd_workspace_size(int64_t n, int32_t c_in, int32_t c_out, int32_t rank) {
+  if (n < 1 || c_in < 1 || c_out < 1 || rank < 1) return 0;
+  return lora_ws(n, c_in, c_out, rank).total;
+}
+
+radial_status radial_lora_bwd(int64_t n, int32_t c_in, int32_t c_out, int32_t rank, float scale, const void* dy,
+                              int64_t lddy, const void* x, int64_t ldx, const void* W, const void* A, const void* B,
+                              const void* u, void* dx, int64_t lddx, int32_t accumulate_dx, void* dA, void* dB,
+                              void* workspace, size_t workspace_bytes, void* stream) {
+  NvtxRange nvtx_range("radial_lora_bwd");
+  radial_status rs = check_lora(n, c_in, c_out, rank, lddy, ldx);
+  if (rs != RADIAL_OK) return rs;
+  if (lddx % 8) return fail(RADIAL_EINVAL, "row strides must be multiples of 8 elements");
+  if (!dy || !x || !W || !A || !B || !u || !dx || !dA || !dB || !workspace)
+    return fail(RADIAL_EINVAL, "NULL pointer");
+  if (!aligned16(dy) || !aligned16(x) || !aligned16(W) || !aligned16(A) || !aligned16(B) || !aligned16(u) ||
+      !aligned16(dx) || !aligned16(dA) || !aligned16(dB))
+    return fail(RADIAL_EINVAL, "pointers must be 16-byte aligned");
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return fail(RADIAL_EINVAL, "workspace must be 256-byte aligned");
+  if (lddy < c_out || ldx < c_in || lddx < c_in) return fail(RADIAL_EINVAL, "row strides must cover the rows");
+  if (accumulate_dx != 0 && accumulate_dx != 1) return fail(RADIAL_EINVAL, "accumulate_dx must be 0 or 1");
+  const LoraWs w = lora_ws(n, c_in, c_out, rank);
+  if (workspace_bytes < w.total)
+    return fail(RADIAL_EINVAL, "workspace of %zu bytes is below the %zu required", workspace_bytes, w.total);
+  cudaStream_t st = as_stream(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  const int64_t ln = pad8(n);
+  void* Wt = ws + w.wt;
+  void* Bt = ws + w.bt;
+  void* At = ws + w.at;
+  void* v = ws + w.v;
+  void* vt = ws + w.vt;
+  void* xt = ws + w.xt;
+  void* dyt = ws + w.dyt;
+  void* ut = ws + w.ut;
+  float* dA32 = reinterpret_cast<float*>(ws + w.dA);
+  float* dB32 = reinterpret_cast<float*>(ws + w.dB);
+  GemmSeg none{nullptr, 0, nullptr, 0, 0};
+  // operands in the orientation the GEMM reads (K contiguous)
+  if ((rs = launch_transpose(W, c_in, c_out, c_in, Wt, c_out, st)) != RADIAL_OK) return rs;    // W^T [ci, co]
+  if ((rs = launch_transpose(B, rank, c_out, rank, Bt, c_out, st)) != RADIAL_OK) return rs;    // B^T [r, co]
+  if ((rs = launch_transpose(A, c_in, rank, c_in, At, rank, st)) != RADIAL_OK) return rs;      // A^T [ci, r]
+  // v = s dy B  [n, r]
+  if ((rs = launch_gemm(n, rank, GemmSeg{dy, lddy, Bt, c_out, c_out}, none, scale, 0.f, v, nullptr, rank, 1, st)) !=
+      RADIAL_OK)
+    return rs;
+  // dx (+)= dy W + v A  [n, ci]
+  if ((rs = launch_gemm(n, c_in, GemmSeg{dy, lddy, Wt, c_out, c_out}, GemmSeg{v, rank, At, rank, rank}, 1.f,
+                        accumulate_dx ? 1.f : 0.f, dx, nullptr, lddx, 1, st)) != RADIAL_OK)
+    return rs;
+  // dA = v^T x  [r, ci] and dB = dy^T u  [co, r]: contractions over all n tokens, split over K
+  if ((rs = launch_transpose(v, rank, n, rank, vt, ln, st)) != RADIAL_OK) return rs;
+  if ((rs = launch_transpose(x, ldx, n, c_in, xt, ln, st)) != RADIAL_OK) return rs;
+  if ((rs = launch_transpose(dy, lddy, n, c_out, dyt, ln, st)) != RADIAL_OK) return rs;
+  if ((rs = launch_transpose(u, rank, n, rank, ut, ln, st)) != RADIAL_OK) return rs;
+  RADIAL_CUDA(cudaMemsetAsync(dA32, 0, sizeof(float) * rank * c_in, st));
+  RADIAL_CUDA(cudaMemsetAsync(dB32, 0, sizeof(float) * c_out * rank, st));
+  if ((rs = launch_gemm(rank, c_in, GemmSeg{vt, ln, xt, ln, n}, none, 1.f, 0.f, nullptr, dA32, c_in, 64, st)) !=
+      RADIAL_OK)
+    return rs;
+  if ((rs = launch_gemm(c_out, rank, GemmSeg{dyt, ln, ut, ln, n}, none, 1.f, 0.f, nullptr, dB32, rank, 64, st)) !=
+      RADIAL_OK)
+    return rs;
+  const int64_t na = static_cast<int64_t>(rank) * c_in, nb = static_cast<int64_t>(c_out) * rank;
+  f32_to_bf16_kernel<<<static_cast<unsigned>((na + 255) / 256), 256, 0, st>>>(dA32, reinterpret_cast<__nv_bfloat16*>(dA), na);
+  RADIAL_LAUNCHED();
+  f32_to_bf16_kernel<<<static_cast<unsigned>((nb + 255) / 256), 256, 0, st>>>(dB32, reinterpret_cast<__nv_bfloat16*>(dB), nb);
+  RADIAL_LAUNCHED();
+  return RADIAL_OK;
+}
 
 }  // extern "C"

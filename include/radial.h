@@ -205,6 +205,41 @@ radial_status radial_attn_bwd_noalloc(const radial_csr* csr, const radial_desc* 
                                       const void* q, const void* k, const void* v, const void* o,
                                       const float* lse, void* dq, void* dk, void* dv, void* stream);
 
+/* ---- LoRA-adapted projections (the fine-tuning layer step around the attention)
+ * The review's §4.3 extends a pretrained video model to longer videos by
+ * training LoRA adapters on the Q/K/V/O projections of its attention layers
+ * while the attention runs under the radial mask.  One projection is
+ *     y = x W^T + s (x A^T) B^T
+ * with W [c_out, c_in] frozen and A [rank, c_in], B [c_out, rank] trained;
+ * the pages fix nothing else, and this standard form, with no bias, is the
+ * reading taken.  All matrices are bf16, row-major with unit column stride;
+ * x, y, dy, dx take a row stride (elements), W, A, B, u, dA, dB are
+ * contiguous.  c_in, c_out, rank and every row stride must be multiples of 8,
+ * every pointer 16-byte aligned.  The GEMMs run on the tensor cores of this
+ * library (fp32 accumulation).  Asynchronous on `stream`; errors as above. */
+
+/* Forward: writes y [n, c_out] and u = s x A^T [n, rank] (bf16), which the
+ * backward takes back. */
+radial_status radial_lora_fwd(int64_t n_tokens, int32_t c_in, int32_t c_out, int32_t rank, float scale,
+                              const void* x, int64_t ldx, const void* W, const void* A, const void* B,
+                              void* y, int64_t ldy, void* u, void* stream);
+
+/* Bytes of device workspace radial_lora_bwd needs (transposed operands and
+ * fp32 accumulators of the adapter gradients).  Host only. */
+size_t radial_lora_bwd_workspace_size(int64_t n_tokens, int32_t c_in, int32_t c_out, int32_t rank);
+
+/* Backward for upstream dy [n, c_out]: dx [n, c_in] = dy W + s (dy B) A
+ * (added to the existing dx when accumulate_dx is 1, so the q, k and v
+ * projections of one input can share a dx), dA [rank, c_in] = s (dy B)^T x
+ * and dB [c_out, rank] = dy^T u (u from the forward).  `workspace`:
+ * caller-owned device memory of radial_lora_bwd_workspace_size bytes,
+ * 256-byte aligned. */
+radial_status radial_lora_bwd(int64_t n_tokens, int32_t c_in, int32_t c_out, int32_t rank, float scale,
+                              const void* dy, int64_t lddy, const void* x, int64_t ldx, const void* W,
+                              const void* A, const void* B, const void* u, void* dx, int64_t lddx,
+                              int32_t accumulate_dx, void* dA, void* dB, void* workspace,
+                              size_t workspace_bytes, void* stream);
+
 /* Synchronise `stream` and report whether any kernel of this library aborted
  * on a bounded wait since the last call (RADIAL_EDEVICE, then cleared), or a
  * CUDA error is pending (RADIAL_ECUDA).  RADIAL_OK otherwise. */

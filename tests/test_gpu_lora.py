@@ -1,10 +1,12 @@
 """LoRA-adapted attention layer step (block_sparse_attention_csr_b200.lora):
-projections in cuBLAS, radial attention in the library's kernels, against the
-fp64 layer reference (oracle.lora) on the same seeded bf16 inputs.
+projections on the library's tensor-core GEMM, radial attention in its
+block-sparse kernels, all through the C ABI, against the fp64 layer
+reference (oracle.lora) on the same seeded bf16 inputs.
 
 The reference rounds to bf16 exactly where the device stores bf16 between
 stages (q, k, v, the attention output, dO), so the remaining differences are
-fp32-accumulated GEMMs and the attention kernels' own error.  Tolerances,
+fp32-accumulated GEMMs, the bf16 low-rank intermediates and the attention
+kernels' own error.  Tolerances,
 relative to the largest reference magnitude of each tensor: max-abs 3e-2 and
 mean-abs 3e-3 -- the attention's own bounds (2e-2 / 2e-3 on unit-scale O,
 5e-2 on gradients) after one more bf16 GEMM stage (relative rounding 2^-9

@@ -1,12 +1,17 @@
-"""Host-side check of the LoRA layer's projection algebra
-(block_sparse_attention_csr_b200.lora): the GEMM sequences of one adapted
-projection and of its backward, run here on CPU float64 tensors, against the
-fp64 layer reference.  (The attention between the projections needs the GPU
-library; its parity is tests/test_gpu_lora.py.)"""
+"""Host-side checks of the LoRA layer (block_sparse_attention_csr_b200.lora)
+and of its projection entry points: the head view of the projection outputs,
+the ABI's argument validation (which rejects before any device work, so it
+runs without a GPU) and the backward's workspace size.  The projections
+themselves run on the library's tensor-core GEMM; their parity against the
+fp64 reference is tests/test_gpu_gemm.py and tests/test_gpu_lora.py."""
+
+import ctypes
 
 import numpy as np
 import torch
 
+from block_sparse_attention_csr_b200 import _binding as B
+from block_sparse_attention_csr_b200 import build as build_mod
 from block_sparse_attention_csr_b200.lora import RadialLoRALayer
 from oracle import lora as LO
 
@@ -20,21 +25,32 @@ def _layer(rng, C, r, s):
     return RadialLoRALayer(None, 4, W, AB, s), W, AB
 
 
-def test_projection_and_backward_match_reference():
-    rng = np.random.default_rng(3)
-    C, r, n, s = 32, 4, 17, 0.375
-    layer, W, AB = _layer(rng, C, r, s)
-    x = torch.tensor(rng.standard_normal((n, C)))
-    dy = torch.tensor(rng.standard_normal((n, C)))
-    for p in LO.PROJ:
-        Wp, Ap, Bp = W["W_" + p].numpy(), AB["A_" + p].numpy(), AB["B_" + p].numpy()
-        np.testing.assert_allclose(layer._proj(x, p).numpy(), LO.lora_linear(x.numpy(), Wp, Ap, Bp, s),
-                                   rtol=1e-12, atol=1e-12)
-        dx, dA, dB = layer._proj_backward(x, p, dy)
-        rdx, rdA, rdB = LO.lora_linear_backward(x.numpy(), Wp, Ap, Bp, s, dy.numpy())
-        np.testing.assert_allclose(dx.numpy(), rdx, rtol=1e-12, atol=1e-11)
-        np.testing.assert_allclose(dA.numpy(), rdA, rtol=1e-12, atol=1e-11)
-        np.testing.assert_allclose(dB.numpy(), rdB, rtol=1e-12, atol=1e-11)
+def _lib():
+    build_mod.build()
+    return B.load()
+
+
+def test_projection_arguments_are_validated_on_the_host():
+    L = _lib()
+    vp = ctypes.c_void_p
+    nul = vp(0)
+    # rank not a multiple of 8, bad sizes, null pointers: EINVAL before any device work
+    assert L.radial_lora_fwd(100, 128, 128, 12, 1.0, nul, 128, nul, nul, nul, nul, 128, nul, None) == 1
+    assert L.radial_lora_fwd(0, 128, 128, 16, 1.0, nul, 128, nul, nul, nul, nul, 128, nul, None) == 1
+    assert L.radial_lora_fwd(100, 128, 128, 16, 1.0, nul, 128, nul, nul, nul, nul, 128, nul, None) == 1
+    assert b"NULL" in L.radial_last_error()
+    assert L.radial_lora_bwd(100, 128, 128, 16, 1.0, nul, 128, nul, 128, nul, nul, nul, nul, nul, 128, 2,
+                             nul, nul, nul, ctypes.c_size_t(0), None) == 1
+
+
+def test_backward_workspace_size():
+    L = _lib()
+    n, ci, co, r = 118800, 3072, 3072, 64
+    got = L.radial_lora_bwd_workspace_size(n, ci, co, r)
+    # transposed W, B, A, v, x, dy, u (bf16) and fp32 dA, dB accumulators
+    need = 2 * (ci * co + r * co + ci * r + n * r + r * n + ci * n + co * n + r * n) + 4 * (r * ci + co * r)
+    assert need <= got <= need + 10 * 256
+    assert L.radial_lora_bwd_workspace_size(0, ci, co, r) == 0
 
 
 def test_head_view_is_the_channel_split():
