@@ -355,15 +355,27 @@ def run_ours(args, rank, world, local_rank):
     # ---- end to end through the public API with host buffers
     e2e = None
     if rank == 0 and not args.quick and local_heads > 0:
-        hq, hk, hv = (t.cpu().pin_memory() for t in (q, k, v))
+        def pinned_like(t):
+            h = torch.empty_strided(t.shape, t.stride(), dtype=t.dtype, pin_memory=True)
+            h.copy_(t)
+            return h
+
+        hq, hk, hv = (pinned_like(t) for t in (q, k, v))
         hdo = do.cpu().pin_memory() if backward else None
-        ho = torch.empty(q.shape, dtype=torch.bfloat16).pin_memory()
+        ho = torch.empty_strided(q.shape, q.stride(), dtype=torch.bfloat16, pin_memory=True)
         hl = torch.empty(q.shape[:3], dtype=torch.float32).pin_memory()
         if backward:
             hdq = torch.empty(q.shape, dtype=torch.bfloat16).pin_memory()
             hdk, hdv = torch.empty_like(hdq).pin_memory(), torch.empty_like(hdq).pin_memory()
 
         def e2e_step():
+            if not backward:
+                # the public host-buffer call: each group of heads is copied in
+                # while the previous group's attention runs, and copied out
+                # while the next one runs
+                rb.radial_attn_fwd_staged(csr, hq, hk, hv, q, k, v, o_host=ho, lse_host=hl, o_dev=o, lse_dev=lse,
+                                          chunks=args.e2e_chunks, stream=stream)
+                return
             q.copy_(hq, non_blocking=True)
             k.copy_(hk, non_blocking=True)
             v.copy_(hv, non_blocking=True)
@@ -395,8 +407,9 @@ def run_ours(args, rank, world, local_rank):
         e2e = {"value": (flops_step if not heads_mode else flops_step * wl.heads / local_heads) / (e2e_ms * 1e-3) / 1e12,
                "unit": "TFLOP/s", "ms_per_step": e2e_ms,
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
-               "path": "pinned host -> device copies, radial_attn_fwd%s via the C ABI, device -> host result copies"
-                       % ("/bwd" if backward else "")}
+               "path": ("pinned host buffers -> radial_attn_fwd_staged (C ABI): H2D copies, attention and D2H copies "
+                        "of %d head groups overlapped" % args.e2e_chunks) if not backward else
+                       "pinned host -> device copies, radial_attn_fwd/bwd via the C ABI, device -> host result copies"}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -596,6 +609,7 @@ def main():
     ap.add_argument("--lora-rank", type=int, default=64)
     ap.add_argument("--step", default=None, choices=["fwd", "bwd", "fwdbwd"],
                     help="what one step runs (default: the workload's own: forward, or forward+backward)")
+    ap.add_argument("--e2e-chunks", type=int, default=6, help="head groups of the staged host-buffer forward")
     ap.add_argument("--shard", default="heads", choices=["heads", "replica"],
                     help="multi-GPU: split the problem's heads across ranks (default) or run one replica per rank")
     args = ap.parse_args()

@@ -16,6 +16,7 @@ from ._binding import (  # noqa: F401
     radial_attn_bwd_noalloc,
     radial_attn_bwd_workspace_size,
     radial_attn_fwd,
+    radial_attn_fwd_staged,
     radial_csr_copy_to_host,
     radial_csr_info,
     radial_device_status,

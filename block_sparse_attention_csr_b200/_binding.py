@@ -30,7 +30,7 @@ EXPORTED = (
     "radial_csr_copy_to_host", "radial_csr_free", "radial_attn_fwd",
     "radial_attn_bwd_workspace_size", "radial_attn_bwd", "radial_device_status",
     "radial_status_str", "radial_last_error", "radial_launch_count", "radial_selftest_bounded_wait",
-    "radial_attn_bwd_noalloc", "radial_lora_fwd", "radial_lora_bwd_workspace_size", "radial_lora_bwd",
+    "radial_attn_bwd_noalloc", "radial_attn_fwd_staged", "radial_lora_fwd", "radial_lora_bwd_workspace_size", "radial_lora_bwd",
 )
 
 
@@ -91,6 +91,8 @@ def load(path=None):
         L.radial_csr_free.restype = None
         L.radial_attn_fwd.argtypes = [vp, ctypes.POINTER(radial_desc)] + [vp] * 6
         L.radial_attn_fwd.restype = ctypes.c_int
+        L.radial_attn_fwd_staged.argtypes = [vp, ctypes.POINTER(radial_desc)] + [vp] * 10 + [i32, vp]
+        L.radial_attn_fwd_staged.restype = ctypes.c_int
         L.radial_attn_bwd_workspace_size.argtypes = [ctypes.POINTER(radial_desc)]
         L.radial_attn_bwd_workspace_size.restype = sz
         L.radial_attn_bwd.argtypes = [vp, ctypes.POINTER(radial_desc)] + [vp] * 10 + [sz, vp]
@@ -246,6 +248,33 @@ def radial_attn_fwd(csr, q, k, v, o=None, lse=None, scale=None, stream=None):
     _check(load().radial_attn_fwd(csr.handle, ctypes.byref(desc), _ptr(q), _ptr(k), _ptr(v), _ptr(o),
                                   _ptr(lse), _stream(stream)), "radial_attn_fwd")
     return o, lse
+
+
+def radial_attn_fwd_staged(csr, q_host, k_host, v_host, q_dev, k_dev, v_dev, o_host=None, lse_host=None,
+                           o_dev=None, lse_dev=None, chunks=4, scale=None, stream=None):
+    """Forward of host (pinned) tensors with the copies overlapped with the
+    attention, group of heads by group of heads.  Host and device tensors
+    share one [B, H, N, D] layout; the outputs land in o_host / lse_host
+    (allocated pinned when not given).  Returns (o_host, lse_host)."""
+    import torch
+    if o_host is None:
+        o_host = torch.empty_strided(q_host.shape, q_host.stride(), dtype=torch.bfloat16).pin_memory()
+    if lse_host is None:
+        lse_host = torch.empty(q_host.shape[:3], dtype=torch.float32).pin_memory()
+    if o_dev is None:
+        o_dev = torch.empty_like(q_dev)
+    if lse_dev is None:
+        lse_dev = torch.empty(q_dev.shape[:3], dtype=torch.float32, device=q_dev.device)
+    _same_layout(q_dev, k_dev, v_dev, o_dev)
+    for t in (q_host, k_host, v_host, o_host):
+        if t.shape != q_dev.shape or t.stride() != q_dev.stride() or t.dtype != torch.bfloat16 or t.is_cuda:
+            raise ValueError("host tensors must be CPU bf16 with the device tensors' shape and strides")
+    desc = make_desc(q_dev, scale)
+    _check(load().radial_attn_fwd_staged(csr.handle, ctypes.byref(desc), _ptr(q_host), _ptr(k_host), _ptr(v_host),
+                                         _ptr(o_host), _ptr(lse_host), _ptr(q_dev), _ptr(k_dev), _ptr(v_dev),
+                                         _ptr(o_dev), _ptr(lse_dev), int(chunks), _stream(stream)),
+           "radial_attn_fwd_staged")
+    return o_host, lse_host
 
 
 def radial_attn_bwd_workspace_size(q):

@@ -657,6 +657,131 @@ radial_status radial_attn_bwd(const radial_csr* c, const radial_desc* d, const v
 }  // extern "C"
 
 // ---------------------------------------------------------------------------
+// Forward of host-resident tensors with the copies overlapped
+// ---------------------------------------------------------------------------
+namespace {
+
+constexpr int kMaxStageGroups = 64;
+
+// Per device: a copy-in and a copy-out stream and the events that order the
+// groups of one call (created on first use, kept until exit).
+struct StageResources {
+  cudaStream_t in = nullptr, out = nullptr;
+  cudaEvent_t start = nullptr, done = nullptr;
+  cudaEvent_t in_done[kMaxStageGroups] = {}, comp_done[kMaxStageGroups] = {};
+};
+std::mutex g_stage_mu;
+StageResources g_stage[64];
+
+radial_status stage_resources(StageResources** out) {
+  int dev = 0;
+  RADIAL_CUDA(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= 64) return fail(RADIAL_EUNSUPPORTED, "device index %d beyond 63", dev);
+  std::lock_guard<std::mutex> lock(g_stage_mu);
+  StageResources& r = g_stage[dev];
+  if (!r.in) {
+    RADIAL_CUDA(cudaStreamCreateWithFlags(&r.in, cudaStreamNonBlocking));
+    RADIAL_CUDA(cudaStreamCreateWithFlags(&r.out, cudaStreamNonBlocking));
+    RADIAL_CUDA(cudaEventCreateWithFlags(&r.start, cudaEventDisableTiming));
+    RADIAL_CUDA(cudaEventCreateWithFlags(&r.done, cudaEventDisableTiming));
+    for (int i = 0; i < kMaxStageGroups; ++i) {
+      RADIAL_CUDA(cudaEventCreateWithFlags(&r.in_done[i], cudaEventDisableTiming));
+      RADIAL_CUDA(cudaEventCreateWithFlags(&r.comp_done[i], cudaEventDisableTiming));
+    }
+  }
+  *out = &r;
+  return RADIAL_OK;
+}
+
+// Copy heads [h0, h1) of batch entry b of one bf16 [B, H, N, D] tensor.
+radial_status copy_heads(void* dst, const void* src, const radial_desc& d, int b, int h0, int h1, cudaMemcpyKind kind,
+                         cudaStream_t st) {
+  const int64_t off = static_cast<int64_t>(b) * d.stride_b + static_cast<int64_t>(h0) * d.stride_h;
+  char* dp = static_cast<char*>(dst) + 2 * off;
+  const char* sp = static_cast<const char*>(src) + 2 * off;
+  if (d.stride_n == d.head_dim && d.stride_h == static_cast<int64_t>(d.n_tokens) * d.head_dim) {
+    // heads of one batch entry are one contiguous block
+    RADIAL_CUDA(cudaMemcpyAsync(dp, sp, static_cast<size_t>(h1 - h0) * d.stride_h * 2, kind, st));
+    return RADIAL_OK;
+  }
+  for (int h = h0; h < h1; ++h) {
+    const int64_t ho = static_cast<int64_t>(h - h0) * d.stride_h * 2;
+    RADIAL_CUDA(cudaMemcpy2DAsync(dp + ho, d.stride_n * 2, sp + ho, d.stride_n * 2, static_cast<size_t>(d.head_dim) * 2,
+                                  static_cast<size_t>(d.n_tokens), kind, st));
+  }
+  return RADIAL_OK;
+}
+
+}  // namespace
+
+extern "C" radial_status radial_attn_fwd_staged(const radial_csr* c, const radial_desc* d, const void* q_host,
+                                                const void* k_host, const void* v_host, void* o_host,
+                                                float* lse_host, void* q_dev, void* k_dev, void* v_dev, void* o_dev,
+                                                float* lse_dev, int32_t chunks, void* stream) {
+  NvtxRange nvtx_range("radial_attn_fwd_staged");
+  radial_status rs = check_desc(c, d);
+  if (rs != RADIAL_OK) return rs;
+  if (!q_host || !k_host || !v_host || !o_host || !lse_host || !q_dev || !k_dev || !v_dev || !o_dev || !lse_dev)
+    return fail(RADIAL_EINVAL, "NULL tensor pointer");
+  if (!aligned16(q_dev) || !aligned16(k_dev) || !aligned16(v_dev) || !aligned16(o_dev) || !aligned16(lse_dev))
+    return fail(RADIAL_EINVAL, "device tensor pointers must be 16-byte aligned");
+  if (chunks < 1) return fail(RADIAL_EINVAL, "chunks must be >= 1");
+  const int per_b = std::min(chunks, d->heads);
+  const int64_t groups = static_cast<int64_t>(d->batch) * per_b;
+  if (groups > kMaxStageGroups)
+    return fail(RADIAL_EUNSUPPORTED, "batch * chunks = %lld exceeds %d groups", (long long)groups, kMaxStageGroups);
+  {
+    // the maps of every group are subsets of these: if they encode, so do
+    // the groups', and no failure can come after the first copy
+    CUtensorMap probe;
+    if ((rs = make_bhnd_map(&probe, q_dev, *d)) != RADIAL_OK) return rs;
+    if ((rs = make_bhnd_map(&probe, k_dev, *d)) != RADIAL_OK) return rs;
+    if ((rs = make_bhnd_map(&probe, v_dev, *d)) != RADIAL_OK) return rs;
+  }
+  StageResources* R = nullptr;
+  if ((rs = stage_resources(&R)) != RADIAL_OK) return rs;
+  cudaStream_t st = as_stream(stream);
+  // nothing on `stream` before this call may still be using the device buffers
+  RADIAL_CUDA(cudaEventRecord(R->start, st));
+  RADIAL_CUDA(cudaStreamWaitEvent(R->in, R->start, 0));
+  RADIAL_CUDA(cudaStreamWaitEvent(R->out, R->start, 0));
+  int g = 0;
+  for (int b = 0; b < d->batch; ++b) {
+    for (int k = 0; k < per_b; ++k, ++g) {
+      const int h0 = k * d->heads / per_b, h1 = (k + 1) * d->heads / per_b;
+      // copy in
+      if ((rs = copy_heads(q_dev, q_host, *d, b, h0, h1, cudaMemcpyHostToDevice, R->in)) != RADIAL_OK) return rs;
+      if ((rs = copy_heads(k_dev, k_host, *d, b, h0, h1, cudaMemcpyHostToDevice, R->in)) != RADIAL_OK) return rs;
+      if ((rs = copy_heads(v_dev, v_host, *d, b, h0, h1, cudaMemcpyHostToDevice, R->in)) != RADIAL_OK) return rs;
+      RADIAL_CUDA(cudaEventRecord(R->in_done[g], R->in));
+      // attention of this group on the caller's stream
+      RADIAL_CUDA(cudaStreamWaitEvent(st, R->in_done[g], 0));
+      radial_desc sub = *d;
+      sub.batch = 1;
+      sub.heads = h1 - h0;
+      const int64_t off = static_cast<int64_t>(b) * d->stride_b + static_cast<int64_t>(h0) * d->stride_h;
+      const int64_t loff = (static_cast<int64_t>(b) * d->heads + h0) * d->n_tokens;
+      const char* qp = static_cast<const char*>(q_dev) + 2 * off;
+      const char* kp = static_cast<const char*>(k_dev) + 2 * off;
+      const char* vp = static_cast<const char*>(v_dev) + 2 * off;
+      char* op = static_cast<char*>(o_dev) + 2 * off;
+      rs = d->head_dim == 128 ? launch_fwd_pair<128>(c, &sub, qp, kp, vp, op, lse_dev + loff, st)
+                              : launch_fwd_pair<64>(c, &sub, qp, kp, vp, op, lse_dev + loff, st);
+      if (rs != RADIAL_OK) return rs;
+      RADIAL_CUDA(cudaEventRecord(R->comp_done[g], st));
+      // copy out
+      RADIAL_CUDA(cudaStreamWaitEvent(R->out, R->comp_done[g], 0));
+      if ((rs = copy_heads(o_host, o_dev, *d, b, h0, h1, cudaMemcpyDeviceToHost, R->out)) != RADIAL_OK) return rs;
+      RADIAL_CUDA(cudaMemcpyAsync(lse_host + loff, lse_dev + loff, sizeof(float) * (h1 - h0) * d->n_tokens,
+                                  cudaMemcpyDeviceToHost, R->out));
+    }
+  }
+  RADIAL_CUDA(cudaEventRecord(R->done, R->out));
+  RADIAL_CUDA(cudaStreamWaitEvent(st, R->done, 0));
+  return RADIAL_OK;
+}
+
+// ---------------------------------------------------------------------------
 // Backward without any allocation: the row-sum scratch lives in a fixed
 // device array of this module instead of a caller-provided workspace.
 // ---------------------------------------------------------------------------

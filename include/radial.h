@@ -162,6 +162,26 @@ typedef struct radial_desc {
 radial_status radial_attn_fwd(const radial_csr* csr, const radial_desc* desc, const void* q,
                               const void* k, const void* v, void* o, float* lse, void* stream);
 
+/* Forward of host-resident tensors with the copies overlapped: the same
+ * result as copying Q, K, V to the device, calling radial_attn_fwd and copying
+ * O and LSE back, but the heads of each batch entry are processed in `chunks`
+ * groups (at most batch * chunks = 64 groups), and group g's inputs are copied
+ * in while group g-1 is computed and group g-1's outputs copied out, on two
+ * internal streams per device created on the first call.  q_host .. lse_host
+ * are host buffers, q_dev .. lse_dev caller-owned device buffers of the full
+ * shape; host and device tensors share the layout of `desc`.  The host
+ * buffers should be page-locked, or the copies cannot overlap.  Work already
+ * queued on `stream` completes before the first copy; `stream` then waits
+ * for the last one, so a synchronisation of `stream` covers the whole call.
+ * All arguments are validated before the first copy; a CUDA error in a copy
+ * itself is reported as RADIAL_ECUDA after earlier groups were issued.  Two
+ * calls on one device at once share the internal streams and run one after
+ * the other.  Asynchronous. */
+radial_status radial_attn_fwd_staged(const radial_csr* csr, const radial_desc* desc, const void* q_host,
+                                     const void* k_host, const void* v_host, void* o_host, float* lse_host,
+                                     void* q_dev, void* k_dev, void* v_dev, void* o_dev, float* lse_dev,
+                                     int32_t chunks, void* stream);
+
 /* Bytes of device workspace radial_attn_bwd needs for this shape: one fp32
  * per (batch, head, token) for the row sums rowsum(dO o O), rounded up to
  * 256 bytes.  Returns 0 for a NULL or empty desc.  Host only. */

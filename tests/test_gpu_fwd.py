@@ -166,3 +166,26 @@ def test_many_work_items_all_rows():
     res = oracle_pool.run("fwd_rows", tasks)
     _check(o[0].float().cpu().numpy().reshape(-1, 128), lse[0].cpu().numpy().reshape(-1),
            np.concatenate([a for a, _ in res]), np.concatenate([b for _, b in res]), "many items")
+
+
+@pytest.mark.parametrize("Bn,H,chunks,permuted", [(1, 5, 3, False), (2, 4, 4, False), (1, 6, 2, True)])
+def test_staged_forward_equals_device_forward(Bn, H, chunks, permuted):
+    """radial_attn_fwd_staged (host buffers, copies overlapped with the
+    attention group by group) gives bit for bit the device call's O and LSE:
+    the same kernel runs on each group of heads.  `permuted` stores
+    [B, N, H, D] viewed as [B, H, N, D], whose heads are not contiguous."""
+    g = torch.Generator(device="cpu").manual_seed(31 + H)
+    N, D, f, s = 1000, 128, 5, 200
+    shape = (Bn, N, H, D) if permuted else (Bn, H, N, D)
+    view = (lambda t: t.permute(0, 2, 1, 3)) if permuted else (lambda t: t)
+    base = [torch.randn(shape, generator=g).to(torch.bfloat16) for _ in range(3)]
+    host = [view(t.pin_memory()) for t in base]
+    dev = [view(t.to(DEV)) for t in base]
+    csr = rb.radial_mask_build(f, s, 128, sink=1)
+    o_ref, l_ref = rb.radial_attn_fwd(csr, *dev)
+    o_dev = view(torch.empty(shape, dtype=torch.bfloat16, device=DEV))
+    o_host = view(torch.empty(shape, dtype=torch.bfloat16).pin_memory())
+    o_h, l_h = rb.radial_attn_fwd_staged(csr, *host, *dev, o_host=o_host, o_dev=o_dev, chunks=chunks)
+    torch.cuda.synchronize()
+    rb.radial_device_status()
+    assert torch.equal(o_h, o_ref.cpu()) and torch.equal(l_h, l_ref.cpu())
