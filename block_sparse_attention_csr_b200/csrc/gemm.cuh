@@ -11,11 +11,13 @@
 // v projections), or an fp32 accumulate-add used by split-K (the adapter
 // gradients contract over all tokens).
 //
-// Tiles of 128 x 128 outputs, K in blocks of 64 (one 128-byte swizzle box);
-// a persistent grid walks (M tile, N tile, K split) items.
+// Tiles of 128 x BN outputs (BN = 256 for wide outputs, 128 otherwise), K in
+// blocks of 64 (one 128-byte swizzle box); a persistent grid walks (M tile,
+// N tile, K split) items.
 // Warp roles (256 threads): warp 0 TMA producer (4-stage ring of A and B
-// boxes); warp 1 TMEM allocation and single-thread MMA issue into one of two
-// accumulators (so the epilogue of one item overlaps the next item's MMAs);
+// boxes); warp 1 TMEM allocation and single-thread MMA issue (M = 128,
+// N = BN) into one of two accumulators (so the epilogue of one item overlaps
+// the next item's MMAs);
 // warps 4-7 the epilogue, one thread per output row (TMEM lane).
 // Rows or columns past M, N read as zeros (TMA) and are not stored; K past a
 // segment's end reads as zeros.
@@ -40,28 +42,33 @@ struct GemmParams {
   int64_t ldc;       // elements
 };
 
+template <int BN>
 struct GemmCfg {
+  static_assert(BN == 128 || BN == 256, "output tile width");
   static constexpr int STAGES = 4;
-  static constexpr int BOX_BYTES = 128 * 64 * 2;  // 128 rows x 64 K, bf16
+  static constexpr int A_BYTES = 128 * 64 * 2;  // 128 rows x 64 K, bf16
+  static constexpr int B_BYTES = BN * 64 * 2;   // BN rows x 64 K
   static constexpr int SMEM_A = 0;
-  static constexpr int SMEM_B = STAGES * BOX_BYTES;
-  static constexpr int SMEM_BAR = 2 * STAGES * BOX_BYTES;
+  static constexpr int SMEM_B = STAGES * A_BYTES;
+  static constexpr int SMEM_BAR = SMEM_B + STAGES * B_BYTES;
   static constexpr int SMEM_BYTES = SMEM_BAR + 256 + 1024;
+  static constexpr uint32_t TMEM_COLS = 2 * BN;  // two accumulators
 };
 
 struct GemmBars {
-  uint64_t full[GemmCfg::STAGES], empty[GemmCfg::STAGES];
+  uint64_t full[4], empty[4];
   uint64_t acc_full[2], acc_empty[2], mma_done;
   uint32_t tmem_base;
   int abort;
 };
 static_assert(sizeof(GemmBars) <= 256, "gemm barrier area");
 
+template <int BN>
 __global__ void __launch_bounds__(256, 1)
     radial_gemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmB0,
                        const __grid_constant__ CUtensorMap tmA1, const __grid_constant__ CUtensorMap tmB1,
                        const GemmParams p) {
-  using C = GemmCfg;
+  using C = GemmCfg<BN>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -85,7 +92,7 @@ __global__ void __launch_bounds__(256, 1)
     fence_barrier_init();
   }
   if (warp == 1) {
-    tmem_alloc(&bars->tmem_base, 256);
+    tmem_alloc(&bars->tmem_base, C::TMEM_COLS);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -123,11 +130,11 @@ __global__ void __launch_bounds__(256, 1)
             ok = false;
             break;
           }
-          mbar_arrive_expect_tx(&bars->full[st], 2 * C::BOX_BYTES);
+          mbar_arrive_expect_tx(&bars->full[st], C::A_BYTES + C::B_BYTES);
           const bool seg0 = kb < p.kb0;
           const int kx = (seg0 ? kb : kb - p.kb0) * 64;
-          tma_load_2d(sA + st * C::BOX_BYTES, seg0 ? &tmA0 : &tmA1, &bars->full[st], kx, tm * 128);
-          tma_load_2d(sB + st * C::BOX_BYTES, seg0 ? &tmB0 : &tmB1, &bars->full[st], kx, tn * 128);
+          tma_load_2d(sA + st * C::A_BYTES, seg0 ? &tmA0 : &tmA1, &bars->full[st], kx, tm * 128);
+          tma_load_2d(sB + st * C::B_BYTES, seg0 ? &tmB0 : &tmB1, &bars->full[st], kx, tn * BN);
         }
       }
       for (uint32_t x = (kc > C::STAGES ? kc - C::STAGES : 0); x < kc; ++x)
@@ -136,8 +143,8 @@ __global__ void __launch_bounds__(256, 1)
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      constexpr uint32_t idesc = idesc_bf16_f32(128, 128, false, false);
-      constexpr uint64_t kBox = C::BOX_BYTES >> 4;
+      constexpr uint32_t idesc = idesc_bf16_f32(128, BN, false, false);
+      constexpr uint64_t kBoxA = C::A_BYTES >> 4, kBoxB = C::B_BYTES >> 4;
       const uint64_t dA0 = smem_desc(smem_u32(sA), 16, 1024, kSwizzle128B);
       const uint64_t dB0 = smem_desc(smem_u32(sB), 16, 1024, kSwizzle128B);
       uint32_t kc = 0, item_i = 0;
@@ -157,7 +164,7 @@ __global__ void __launch_bounds__(256, 1)
           tc_fence_after();
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
-            mma_ss(tmem + ab * 128, dA0 + st * kBox + ((kk * 32) >> 4), dB0 + st * kBox + ((kk * 32) >> 4), idesc,
+            mma_ss(tmem + ab * BN, dA0 + st * kBoxA + ((kk * 32) >> 4), dB0 + st * kBoxB + ((kk * 32) >> 4), idesc,
                    (kb > kb0 || kk > 0) ? 1u : 0u);
           mma_commit(&bars->empty[st]);
         }
@@ -180,11 +187,11 @@ __global__ void __launch_bounds__(256, 1)
       tc_fence_after();
       const int row = tm * 128 + quarter * 32 + lane;
 #pragma unroll 1
-      for (int c = 0; c < 4; ++c) {
+      for (int c = 0; c < BN / 32; ++c) {
         uint32_t r[32];
-        tmem_ld32(tmem + lane_addr + ab * 128 + c * 32, r);
+        tmem_ld32(tmem + lane_addr + ab * BN + c * 32, r);
         tmem_wait_ld();
-        const int col0 = tn * 128 + c * 32;
+        const int col0 = tn * BN + c * 32;
         if (!waited || row >= p.M || col0 >= p.N) continue;
         if (p.acc) {
           float* dst = p.acc + static_cast<int64_t>(row) * p.ldc + col0;
@@ -223,7 +230,7 @@ __global__ void __launch_bounds__(256, 1)
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, 256);
+    tmem_dealloc(tmem, C::TMEM_COLS);
   }
 }
 

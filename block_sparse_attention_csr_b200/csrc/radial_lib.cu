@@ -898,12 +898,13 @@ namespace {
 
 // 2D map over a bf16 row-major [rows, cols] matrix with row stride ld
 // (elements): 64-column x 128-row boxes, 128-byte swizzle; outside reads 0.
-radial_status make_rowmajor_map(CUtensorMap* map, const void* base, int64_t rows, int64_t cols, int64_t ld) {
+radial_status make_rowmajor_map(CUtensorMap* map, const void* base, int64_t rows, int64_t cols, int64_t ld,
+                                uint32_t box_rows = 128) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return fail(RADIAL_ECUDA, "cuTensorMapEncodeTiled unavailable");
   cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
   cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld) * 2};
-  cuuint32_t box[2] = {64, 128};
+  cuuint32_t box[2] = {64, box_rows};
   cuuint32_t estr[2] = {1, 1};
   CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -921,17 +922,16 @@ struct GemmSeg {
   int64_t k;  // 0: no segment
 };
 
-// C[M, N] = alpha (A0 B0^T + A1 B1^T) + beta C (bf16 c) or acc += ... (fp32,
-// split over K into up to `max_splits` slices).  Encodes every map first.
-radial_status launch_gemm(int64_t M, int64_t N, const GemmSeg& s0, const GemmSeg& s1, float alpha, float beta,
-                          void* c, float* acc, int64_t ldc, int max_splits, cudaStream_t st) {
+template <int BN>
+radial_status launch_gemm_bn(int64_t M, int64_t N, const GemmSeg& s0, const GemmSeg& s1, float alpha, float beta,
+                             void* c, float* acc, int64_t ldc, int max_splits, cudaStream_t st) {
   CUtensorMap a0, b0, a1, b1;
   radial_status rs;
   if ((rs = make_rowmajor_map(&a0, s0.a, M, s0.k, s0.lda)) != RADIAL_OK) return rs;
-  if ((rs = make_rowmajor_map(&b0, s0.b, N, s0.k, s0.ldb)) != RADIAL_OK) return rs;
+  if ((rs = make_rowmajor_map(&b0, s0.b, N, s0.k, s0.ldb, BN)) != RADIAL_OK) return rs;
   if (s1.k > 0) {
     if ((rs = make_rowmajor_map(&a1, s1.a, M, s1.k, s1.lda)) != RADIAL_OK) return rs;
-    if ((rs = make_rowmajor_map(&b1, s1.b, N, s1.k, s1.ldb)) != RADIAL_OK) return rs;
+    if ((rs = make_rowmajor_map(&b1, s1.b, N, s1.k, s1.ldb, BN)) != RADIAL_OK) return rs;
   } else {
     a1 = a0;
     b1 = b0;
@@ -942,7 +942,7 @@ radial_status launch_gemm(int64_t M, int64_t N, const GemmSeg& s0, const GemmSeg
   p.kb0 = static_cast<int32_t>((s0.k + 63) / 64);
   p.kb_total = p.kb0 + static_cast<int32_t>((s1.k + 63) / 64);
   p.tiles_m = static_cast<int32_t>((M + 127) / 128);
-  p.tiles_n = static_cast<int32_t>((N + 127) / 128);
+  p.tiles_n = static_cast<int32_t>((N + BN - 1) / BN);
   const int tiles = p.tiles_m * p.tiles_n;
   int splits = 1;
   if (acc) {  // split K until the grid fills the device
@@ -956,12 +956,22 @@ radial_status launch_gemm(int64_t M, int64_t N, const GemmSeg& s0, const GemmSeg
   p.c = reinterpret_cast<__nv_bfloat16*>(c);
   p.acc = acc;
   p.ldc = ldc;
-  RADIAL_CUDA(cudaFuncSetAttribute(radial_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                   GemmCfg::SMEM_BYTES));
+  RADIAL_CUDA(cudaFuncSetAttribute(radial_gemm_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                   GemmCfg<BN>::SMEM_BYTES));
   const int grid = p.items < sm_count() ? p.items : sm_count();
-  radial_gemm_kernel<<<grid, 256, GemmCfg::SMEM_BYTES, st>>>(a0, b0, a1, b1, p);
+  radial_gemm_kernel<BN><<<grid, 256, GemmCfg<BN>::SMEM_BYTES, st>>>(a0, b0, a1, b1, p);
   RADIAL_LAUNCHED();
   return RADIAL_OK;
+}
+
+// C[M, N] = alpha (A0 B0^T + A1 B1^T) + beta C (bf16 c) or acc += ... (fp32,
+// split over K into up to `max_splits` slices).  Encodes every map first.
+// Output tiles are 128 x 256 when N is wider than 128 (half the MMA
+// instructions and A re-reads of 128 x 128 tiles), else 128 x 128.
+radial_status launch_gemm(int64_t M, int64_t N, const GemmSeg& s0, const GemmSeg& s1, float alpha, float beta,
+                          void* c, float* acc, int64_t ldc, int max_splits, cudaStream_t st) {
+  if (N > 128) return launch_gemm_bn<256>(M, N, s0, s1, alpha, beta, c, acc, ldc, max_splits, st);
+  return launch_gemm_bn<128>(M, N, s0, s1, alpha, beta, c, acc, ldc, max_splits, st);
 }
 
 radial_status launch_transpose(const void* in, int64_t ld_in, int64_t R, int64_t Cc, void* out, int64_t ld_out,
