@@ -95,37 +95,6 @@ struct BwdParams {
   const int32_t* cd;
 };
 
-// Allowed query rows (relative to a0, 128 wide) of key token b = j*s + l:
-// the transpose of row_mask_bits.
-__device__ __forceinline__ void col_mask_bits(const int32_t* hd, const int32_t* cd, int s, int n, int sink,
-                                              int j, int l, int a0, uint32_t (&mw)[4]) {
-  mw[0] = mw[1] = mw[2] = mw[3] = 0u;
-  const int aend = min(a0 + 128, n);
-  for (int i = a0 / s; i * s < aend; ++i) {
-    const int seg_lo = max(a0, i * s) - a0;
-    const int seg_hi = min(aend, (i + 1) * s) - 1 - a0;
-    int lo, hi;
-    if (sink && j == 0) {
-      lo = seg_lo;
-      hi = seg_hi;
-    } else {
-      const int d = i > j ? i - j : j - i;
-      const int h = half_width_of(hd, s, d);
-      const int center = i * s + l - a0;
-      if (h >= 0) {
-        lo = max(seg_lo, center - h);
-        hi = min(seg_hi, center + h);
-      } else {
-        const long long period = period_of(cd, s, d);
-        if (d % period != 0) continue;
-        lo = max(seg_lo, center);
-        hi = min(seg_hi, center);
-      }
-    }
-    if (lo <= hi) set_bits(mw, lo, hi);
-  }
-}
-
 template <int D>
 struct BwdCfg {
   static constexpr int TILE_BYTES = 128 * D * 2;
@@ -332,6 +301,13 @@ __global__ void __launch_bounds__(384, 1)
       const bool valid = key < p.n;
       const int kj = valid ? key / p.s : 0;
       const int kl = valid ? key - kj * p.s : 0;
+      RowMaskGeom mg{};
+      mg.f = p.f;
+      mg.s = p.s;
+      mg.n = p.n;
+      mg.sink = p.sink;
+      mg.hd = p.hd;
+      mg.cd = p.cd;
       const int c0 = p.col_ptr[u];
       const uint32_t n_tiles = static_cast<uint32_t>(p.col_ptr[u + 1] - c0);
       const float* lse_bh = p.lse + static_cast<int64_t>(bh) * p.n;
@@ -350,12 +326,12 @@ __global__ void __launch_bounds__(384, 1)
             vbuf[row] = a < p.n ? dr_bh[a] : 0.f;
         }
         named_bar_sync(1 + wg, 128);
-        uint32_t mw[4] = {0xffffffffu, 0xffffffffu, 0xffffffffu, 0xffffffffu};
+        // this warpgroup's 64 queries of the tile, one bit each
+        uint32_t mw[2] = {0xffffffffu, 0xffffffffu};
         if (partial) {
-          if (valid)
-            col_mask_bits(p.hd, p.cd, p.s, p.n, p.sink, kj, kl, t * 128, mw);
-          else
-            mw[0] = mw[1] = mw[2] = mw[3] = 0u;
+          const uint64_t m64 = valid ? col_mask64(mg, kj, kl, t * 128 + 64 * wg) : 0ull;
+          mw[0] = static_cast<uint32_t>(m64);
+          mw[1] = static_cast<uint32_t>(m64 >> 32);
         }
         const uint32_t modes = partial ? chunk_modes(mw) : 0u;
         // pass 1: P^T = exp2(S^T * scale*log2e - lse2), kept in fp32 for pass 2
@@ -366,7 +342,7 @@ __global__ void __launch_bounds__(384, 1)
 #pragma unroll
         for (int c = 0; c < 2; ++c) {
           const int gc = 2 * wg + c;  // 32-column chunk of the tile
-          const uint32_t mode = (modes >> (2 * gc)) & 3u;
+          const uint32_t mode = (modes >> (2 * c)) & 3u;
           uint32_t pw[16];
           if (mode == 2u) {  // every lane of the warp masks this chunk: P^T = 0
 #pragma unroll
@@ -377,7 +353,7 @@ __global__ void __launch_bounds__(384, 1)
             uint32_t rs[32];
             tmem_ld32(tmem + lane_addr + TM_S + gc * 32, rs);
             tmem_wait_ld();
-            const uint32_t bits = mode == 0u ? 0xffffffffu : mw[gc];
+            const uint32_t bits = mode == 0u ? 0xffffffffu : mw[c];
 #pragma unroll
             for (int e = 0; e < 32; ++e) {
               const float x = fmaf(__uint_as_float(rs[e]), p.scale_log2, -vbuf[c * 32 + e]);
@@ -400,7 +376,7 @@ __global__ void __launch_bounds__(384, 1)
 #pragma unroll
         for (int c = 0; c < 2; ++c) {
           const int gc = 2 * wg + c;
-          const uint32_t mode = (modes >> (2 * gc)) & 3u;
+          const uint32_t mode = (modes >> (2 * c)) & 3u;
           uint32_t dw[16];
           if (mode == 2u) {
 #pragma unroll
@@ -612,6 +588,13 @@ __global__ void __launch_bounds__(384, 1)
       const bool valid = a < p.n;
       const int qi = valid ? a / p.s : 0;
       const int qk = valid ? a - qi * p.s : 0;
+      RowMaskGeom mg{};
+      mg.f = p.f;
+      mg.s = p.s;
+      mg.n = p.n;
+      mg.sink = p.sink;
+      mg.hd = p.hd;
+      mg.cd = p.cd;
       const float lse2 = valid ? p.lse[static_cast<int64_t>(bh) * p.n + a] * kLog2e : INFINITY;
       const float drow = valid ? p.dr[static_cast<int64_t>(bh) * p.n + a] : 0.f;
       const int p0 = p.row_ptr[t];
@@ -620,19 +603,12 @@ __global__ void __launch_bounds__(384, 1)
         const uint32_t g = it + j, db = g & 1;
         const int kb = RADIAL_CHECK_INDEX(p.col_idx[p0 + j], 0, p.nt);
         const bool partial = p.kind[p0 + j] != kTileFull;
-        uint32_t mw[4] = {0xffffffffu, 0xffffffffu, 0xffffffffu, 0xffffffffu};
+        // this warpgroup's 64 keys of the tile, one bit each
+        uint32_t mw[2] = {0xffffffffu, 0xffffffffu};
         if (partial) {
-          mw[0] = mw[1] = mw[2] = mw[3] = 0u;
-          if (valid) {
-            RowMaskGeom mp{};
-            mp.f = p.f;
-            mp.s = p.s;
-            mp.n = p.n;
-            mp.sink = p.sink;
-            mp.hd = p.hd;
-            mp.cd = p.cd;
-            row_mask_bits(mp, qi, qk, kb * 128, mw);
-          }
+          const uint64_t m64 = valid ? row_mask64(mg, qi, qk, kb * 128 + 64 * wg) : 0ull;
+          mw[0] = static_cast<uint32_t>(m64);
+          mw[1] = static_cast<uint32_t>(m64 >> 32);
         }
         // dS buffer db was read by the dQ MMA of tile g-2
         if (g >= 2) {
@@ -646,7 +622,7 @@ __global__ void __launch_bounds__(384, 1)
 #pragma unroll
         for (int c = 0; c < 2; ++c) {
           const int gc = 2 * wg + c;
-          const uint32_t mode = (modes >> (2 * gc)) & 3u;
+          const uint32_t mode = (modes >> (2 * c)) & 3u;
           uint32_t dw[16];
           if (mode == 2u) {  // every lane of the warp masks this chunk: dS = 0
 #pragma unroll
@@ -664,7 +640,7 @@ __global__ void __launch_bounds__(384, 1)
               tc_fence_before();
               mbar_arrive(&bars->s_free);
             }
-            const uint32_t bits = mw[gc];
+            const uint32_t bits = mw[c];
 #pragma unroll
             for (int e = 0; e < 16; ++e) {
               float dv[2];

@@ -7,7 +7,7 @@
 // the method runs block-wise on 128x128 token blocks).  The mask's
 // element-level pattern is applied on PARTIAL tiles only: each softmax
 // thread derives the allowed key columns of its query row from the frame
-// segments the key tile spans (row_mask_bits below), and warps skip or keep
+// segments the key tile spans (row_mask64 below), and warps skip or keep
 // whole 32-key chunks when every lane agrees (chunk_modes).  The kernel
 // itself is in attn_fwd_pair.cuh.
 #pragma once
@@ -29,18 +29,6 @@ struct RowMaskGeom {
   const int32_t* cd;
 };
 
-__device__ __forceinline__ void set_bits(uint32_t (&mw)[4], int lo, int hi) {
-#pragma unroll
-  for (int w = 0; w < 4; ++w) {
-    const int wlo = max(lo, 32 * w), whi = min(hi, 32 * w + 31);
-    if (wlo <= whi) {
-      const uint32_t nbits = static_cast<uint32_t>(whi - wlo + 1);
-      const uint32_t bits = (nbits == 32u) ? 0xffffffffu : (((1u << nbits) - 1u) << (wlo - 32 * w));
-      mw[w] |= bits;
-    }
-  }
-}
-
 // floor(x / s) for 0 <= x < 2^30 without an integer division: a float
 // estimate from the reciprocal, then an exact correction of at most one step.
 __device__ __forceinline__ int div_by(int x, int s) {
@@ -50,44 +38,75 @@ __device__ __forceinline__ int div_by(int x, int s) {
   return q;
 }
 
-// Allowed key columns (relative to b0, 128 wide) of query token a = i*s + k.
-__device__ __forceinline__ void row_mask_bits(const RowMaskGeom& p, int i, int k, int b0,
-                                              uint32_t (&mw)[4]) {
-  mw[0] = mw[1] = mw[2] = mw[3] = 0u;
-  const int bend = min(b0 + 128, p.n);  // exclusive
-  for (int j = div_by(b0, p.s); j * p.s < bend; ++j) {
-    const int seg_lo = max(b0, j * p.s) - b0;
-    const int seg_hi = min(bend, (j + 1) * p.s) - 1 - b0;
-    int lo, hi;
-    if (p.sink && j == 0) {
-      lo = seg_lo;
-      hi = seg_hi;
-    } else {
-      const int d = i > j ? i - j : j - i;
-      const int h = half_width_of(p.hd, p.s, d);
-      const int center = j * p.s + k - b0;
-      if (h >= 0) {
-        lo = max(seg_lo, center - h);
-        hi = min(seg_hi, center + h);
-      } else {
-        const long long period = period_of(p.cd, p.s, d);
-        if (d % period != 0) continue;
-        lo = max(seg_lo, center);
-        hi = min(seg_hi, center);
-      }
-    }
-    if (lo <= hi) set_bits(mw, lo, hi);
-  }
+// Bits [lo, hi] of a 64-bit word, 0 <= lo <= hi <= 63.
+__device__ __forceinline__ uint64_t bit_range64(int lo, int hi) {
+  return (~0ull >> (63 - hi)) & (~0ull << lo);
 }
 
-// Warp-uniform handling of one 32-column chunk of a PARTIAL tile: 0 = every
-// lane of the warp allows all 32 columns (use S as is), 2 = every lane masks
-// all of them (no TMEM read, no select, no exponential: P = 0), 1 = mixed
-// (per-element select).  Two bits per chunk.
-__device__ __forceinline__ uint32_t chunk_modes(const uint32_t (&mw)[4]) {
+// Token t = own*s + pos (a query for the row mask, a key for the column mask)
+// against the tokens of frame j held by window columns [lo_s, hi_s] (relative
+// to b0): the band |pos - pos'| <= h(d), or the sampled diagonal, as bits.
+__device__ __forceinline__ uint64_t interval_bits64(const RowMaskGeom& p, int own, int pos, int b0, int j, int lo_s,
+                                                    int hi_s) {
+  const int d = own > j ? own - j : j - own;
+  const int h = half_width_of(p.hd, p.s, d);
+  const int center = j * p.s + pos - b0;
+  int lo, hi;
+  if (h >= 0) {
+    lo = max(lo_s, center - h);
+    hi = min(hi_s, center + h);
+  } else {
+    if (d % period_of(p.cd, p.s, d) != 0) return 0ull;
+    lo = max(lo_s, center);
+    hi = min(hi_s, center);
+  }
+  return lo <= hi ? bit_range64(lo, hi) : 0ull;
+}
+
+// Allowed partners in window [b0, b0 + 64) of token own*s + pos, one word
+// (bit c = token b0 + c; tokens at or past n are not allowed).  kKeys = false:
+// the token is a query and the window holds keys (the sink is key frame 0);
+// kKeys = true: the token is a key and the window holds queries (a key of
+// frame 0 is seen by every query).  With s >= 64 the window holds at most two
+// frame segments, each one interval.
+template <bool kKeys>
+__device__ __forceinline__ uint64_t window_mask64(const RowMaskGeom& p, int own, int pos, int b0) {
+  const int bend = min(b0 + 64, p.n) - b0;  // columns inside the sequence
+  if (bend <= 0) return 0ull;
+  if (kKeys && p.sink && own == 0) return bit_range64(0, bend - 1);
+  auto seg = [&](int j, int lo_s, int hi_s) -> uint64_t {
+    if (!kKeys && p.sink && j == 0) return bit_range64(lo_s, hi_s);
+    return interval_bits64(p, own, pos, b0, j, lo_s, hi_s);
+  };
+  int j = div_by(b0, p.s);
+  if (p.s >= 64) {
+    const int e = (j + 1) * p.s - b0;  // first column of frame j + 1
+    if (e >= bend) return seg(j, 0, bend - 1);
+    return seg(j, 0, e - 1) | seg(j + 1, e, bend - 1);
+  }
+  uint64_t m = 0ull;
+  for (; j * p.s < b0 + bend; ++j) m |= seg(j, max(0, j * p.s - b0), min(bend, (j + 1) * p.s - b0) - 1);
+  return m;
+}
+
+// Allowed keys [b0, b0 + 64) of query token i*s + k.
+__device__ __forceinline__ uint64_t row_mask64(const RowMaskGeom& p, int i, int k, int b0) {
+  return window_mask64<false>(p, i, k, b0);
+}
+
+// Allowed queries [a0, a0 + 64) of key token j*s + l (the transpose).
+__device__ __forceinline__ uint64_t col_mask64(const RowMaskGeom& p, int j, int l, int a0) {
+  return window_mask64<true>(p, j, l, a0);
+}
+
+// Warp-uniform handling of a thread's two 32-column chunks of a PARTIAL tile:
+// 0 = every lane of the warp allows all 32 columns (use S as is), 2 = every
+// lane masks all of them (no TMEM read, no select, no exponential: P = 0),
+// 1 = mixed (per-element select).  Two bits per chunk.
+__device__ __forceinline__ uint32_t chunk_modes(const uint32_t (&mw)[2]) {
   uint32_t modes = 0;
 #pragma unroll
-  for (int c = 0; c < 4; ++c) {
+  for (int c = 0; c < 2; ++c) {
     const bool all_ok = __all_sync(0xffffffffu, mw[c] == 0xffffffffu);
     const bool none = __all_sync(0xffffffffu, mw[c] == 0u);
     modes |= (all_ok ? 0u : (none ? 2u : 1u)) << (2 * c);

@@ -10,7 +10,7 @@
 // shifted by 128 tokens); a key tile only one of them needs is computed for
 // that tile alone.
 //
-// Warp roles (384 threads; at most 168 registers each, 148 used):
+// Warp roles (384 threads; at most 168 registers each, 144 used):
 //   warp 0      TMA producer: Q0, Q1 once per item; K and V through
 //               separate 3-slot / 2-slot rings, K one union column ahead of V.
 //   warps 2-3   idle (keep the softmax warps on warpgroup boundaries).
@@ -23,7 +23,8 @@
 //               S1(u), S0(u+1), ...): warpgroup wg takes key columns
 //               [64 wg, 64 wg + 64), one thread per query row; the two warps
 //               on the same TMEM lane quarter exchange row maxima through
-//               shared memory.  Lazy rescaling, packed fp32x2 math.  The MUFU
+//               double-buffered shared memory, one named barrier per
+//               exchange.  Lazy rescaling, packed fp32x2 math.  The MUFU
 //               (16 exponentials per clock and SM) needs all of the 1024
 //               cycles to exponentiate one 128x128 tile, so one warp per SMSP
 //               and tile left it idle during every TMEM round trip; two warps
@@ -37,7 +38,10 @@
 // issued after PV_i(u) in the same MMA stream and executes after it.
 //
 // Shared memory: Q0, Q1 + 3 K slots + 2 V slots, 128 x D bf16 each, 128-byte
-// swizzle in 64-column boxes (224 KB at D = 128).
+// swizzle in 64-column boxes (224 KB at D = 128), then the barriers and the
+// 2 KB row-exchange buffer: 227 KB, the per-block maximum.  The tiles need a
+// 1024-byte aligned base; a launch whose shared memory base is off by more
+// than the 768 bytes of slack does nothing and records kErrLayout.
 //
 // Work items are (batch*head, pair) in head-major order; within a head the
 // pairs run longest-first when an order array is given (the default), else in
@@ -80,8 +84,12 @@ struct FwdPairCfg {
   static constexpr int SMEM_K = 2 * TILE_BYTES;
   static constexpr int SMEM_V = SMEM_K + K_SLOTS * TILE_BYTES;
   static constexpr int SMEM_BAR = SMEM_V + V_SLOTS * TILE_BYTES;
-  static constexpr int SMEM_X = SMEM_BAR + 256;        // float[2][128] row exchange
-  static constexpr int SMEM_BYTES = SMEM_X + 1024 + 1024;
+  static constexpr int SMEM_X = SMEM_BAR + 256;  // float[2 slots][2 warpgroups][128 rows] row exchange
+  // the tiles need a 1024-byte aligned base; the dynamic shared memory base
+  // is aligned that way in practice, and the kernel checks that its
+  // alignment pad fits this slack before it touches anything
+  static constexpr int ALIGN_SLACK = 768;
+  static constexpr int SMEM_BYTES = SMEM_X + 2048 + ALIGN_SLACK;
   static constexpr uint32_t TM_S = 0, TM_O = 256;
 };
 
@@ -100,8 +108,12 @@ __global__ void __launch_bounds__(384, 1)
                            const __grid_constant__ CUtensorMap tmV, const FwdPairParams p) {
   using C = FwdPairCfg<D>;
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  const uint32_t align_pad = (1024u - (smem_u32(smem_raw) & 1023u)) & 1023u;
+  if (align_pad > static_cast<uint32_t>(C::ALIGN_SLACK)) {  // uniform over the grid: every thread returns
+    if (threadIdx.x == 0) atomicExch(&g_device_error, kErrLayout);
+    return;
+  }
+  uint8_t* smem = smem_raw + align_pad;
   uint8_t* sQ = smem + C::SMEM_Q;
   uint8_t* sK = smem + C::SMEM_K;
   uint8_t* sV = smem + C::SMEM_V;
@@ -282,25 +294,29 @@ __global__ void __launch_bounds__(384, 1)
     // columns [64 wg, 64 wg + 64), warp (wg, quarter) the 32 rows of TMEM
     // lane quarter `quarter`.  The two warps sharing a quarter (same rows,
     // same SMSP) exchange partial row maxima -- and at the end row sums --
-    // through shared memory under a 64-thread named barrier, so both apply
-    // the same running maximum m.  Two warps per SMSP keep the MUFU busy
-    // while one of them waits on TMEM or the exchange.
+    // through shared memory, so both apply the same running maximum m.  Two
+    // warps per SMSP keep the MUFU busy while one of them waits on TMEM.
     const int wg = (warp - 4) >> 2;
     const int quarter = warp & 3;
     const int row = quarter * 32 + lane;
     const uint32_t lane_addr = static_cast<uint32_t>(quarter * 32) << 16;
     const int col0 = wg * 64;
-    float* xchg = reinterpret_cast<float*>(smem + C::SMEM_X);
-    volatile float* x_mine = xchg + wg * 128 + row;
-    volatile float* x_peer = xchg + (1 - wg) * 128 + row;
+    // Exchange k (both warps of a quarter run the same sequence) uses slot
+    // k & 1: xput writes this warp's value; xtake meets the peer at the
+    // quarter's named barrier and reads the peer's value.  One barrier per
+    // exchange: slot k & 1 is written again by exchange k + 2, after the
+    // barrier of exchange k + 1, which the peer reaches only after its read
+    // of exchange k.  (A single slot needs a second barrier before the write;
+    // that version was 5-7 % slower.)
+    volatile float* xchg = reinterpret_cast<volatile float*>(smem + C::SMEM_X);
     const int bar_id = 1 + quarter;
-    // write v, read the peer's: the first barrier guarantees the peer has read
-    // the previous value, the second that it has written this one
-    auto exchange = [&](float v) {
+    uint32_t xk = 0;
+    auto xput = [&](float v) { xchg[(xk & 1u) * 256 + wg * 128 + row] = v; };
+    auto xtake = [&]() {
       named_bar_sync(bar_id, 64);
-      *x_mine = v;
-      named_bar_sync(bar_id, 64);
-      return *x_peer;
+      const float v = xchg[(xk & 1u) * 256 + (1 - wg) * 128 + row];
+      ++xk;
+      return v;
     };
     constexpr float kRescaleThreshold = 8.0f;
     RowMaskGeom mp{};
@@ -349,10 +365,11 @@ __global__ void __launch_bounds__(384, 1)
           tmem_ld32(tm_s + col0 + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
           // the mask bits of a PARTIAL tile are computed while the load is in flight
           const bool part = (fl & (ti == 0 ? kPairPart0 : kPairPart1)) != 0;
-          uint32_t mw[4] = {0xffffffffu, 0xffffffffu, 0xffffffffu, 0xffffffffu};
+          uint32_t mw[2] = {0xffffffffu, 0xffffffffu};
           if (part) {
-            mw[0] = mw[1] = mw[2] = mw[3] = 0u;
-            if (valid[ti]) row_mask_bits(mp, qi[ti], qk[ti], kb * 128 + col0, mw);
+            const uint64_t m64 = valid[ti] ? row_mask64(mp, qi[ti], qk[ti], kb * 128 + col0) : 0ull;
+            mw[0] = static_cast<uint32_t>(m64);
+            mw[1] = static_cast<uint32_t>(m64 >> 32);
           }
           uint32_t live = 3u;  // 32-key chunks with an allowed key in some lane of the warp
           uint32_t mixed = 0u;  // chunks that need the per-element select
@@ -380,51 +397,9 @@ __global__ void __launch_bounds__(384, 1)
             }
           }
           const float mloc = max3f(acc[0], acc[1], fmaxf(acc[2], acc[3]));
-          const float m_tile = fmaxf(mloc, exchange(mloc)) * p.scale_log2;
-          // lazy rescaling: m moves only when the tile's maximum exceeds it by
-          // more than the threshold (P stays below 2^8)
-          const bool grow = m_tile > m[ti] + kRescaleThreshold;
-          const bool resc = !first[ti] && __any_sync(0xffffffffu, grow);
-          const float factor = (grow && !first[ti]) ? ex2_approx(m[ti] - m_tile) : 1.0f;
-          if (grow) {
-            l[ti] *= factor;
-            m[ti] = m_tile;
-          }
-          const float m_use = (m[ti] == -INFINITY) ? 0.f : m[ti];
-          const uint64_t sl2 = f2_pack(p.scale_log2, p.scale_log2);
-          const uint64_t negm = f2_pack(-m_use, -m_use);
-          uint64_t acc2[2] = {0ull, 0ull};
-#pragma unroll
-          for (int c = 0; c < 2; ++c) {
-            uint32_t w[16];
-            if (!(live & (1u << c))) {
-#pragma unroll
-              for (int e = 0; e < 16; ++e) w[e] = 0u;
-              tmem_st16(tm_s + wg * 32 + c * 16, w);
-              continue;
-            }
-#pragma unroll
-            for (int e = 0; e < 16; ++e) {
-              const int k2 = 32 * c + 2 * e;
-              const uint64_t xs = f2_fma(f2_pack(__uint_as_float(r[k2]), __uint_as_float(r[k2 + 1])), sl2, negm);
-              float x0, x1;
-              f2_unpack(xs, x0, x1);
-              const uint64_t pe = f2_pack(ex2_approx(x0), ex2_approx(x1));
-              acc2[e & 1] = f2_add(acc2[e & 1], pe);
-              float p0, p1;
-              f2_unpack(pe, p0, p1);
-              w[e] = pack_bf16x2(p0, p1);
-            }
-            // P (bf16 pairs) of keys [col0 + 32 c, +32) -> TMEM columns (col0 + 32 c) / 2
-            tmem_st16(tm_s + wg * 32 + c * 16, w);
-          }
-          const uint64_t s01 = f2_add(acc2[0], acc2[1]);
-          float s0, s1;
-          f2_unpack(s01, s0, s1);
-          l[ti] += s0 + s1;
-          if (resc) {
-            // O_i holds every earlier PV (the S commit covers them); this
-            // warp rescales its half of the output columns
+          // O_i holds every earlier PV (the S commit covers them); this warp
+          // rescales its half of the output columns
+          auto rescale_o = [&](float factor) {
             const uint32_t tm_o = tmem + lane_addr + C::TM_O + ti * 128 + wg * (D / 2);
 #pragma unroll
             for (int c = 0; c < D / 64; ++c) {
@@ -435,7 +410,57 @@ __global__ void __launch_bounds__(384, 1)
               for (int e = 0; e < 32; ++e) ro[e] = __float_as_uint(__uint_as_float(ro[e]) * factor);
               tmem_st32(tm_o + c * 32, ro);
             }
+          };
+          const uint64_t sl2 = f2_pack(p.scale_log2, p.scale_log2);
+          // P = exp2(S * scale * log2(e) - m) of this warp's 64 keys (bf16
+          // pairs) -> TMEM columns (col0 + 32 c) / 2, over the consumed S;
+          // returns the row's sum of them
+          auto make_p = [&](float m_run) {
+            const float m_use = (m_run == -INFINITY) ? 0.f : m_run;
+            const uint64_t negm = f2_pack(-m_use, -m_use);
+            uint64_t acc2[2] = {0ull, 0ull};
+#pragma unroll
+            for (int c = 0; c < 2; ++c) {
+              uint32_t w[16];
+              if (!(live & (1u << c))) {
+#pragma unroll
+                for (int e = 0; e < 16; ++e) w[e] = 0u;
+                tmem_st16(tm_s + wg * 32 + c * 16, w);
+                continue;
+              }
+#pragma unroll
+              for (int e = 0; e < 16; ++e) {
+                const int k2 = 32 * c + 2 * e;
+                const uint64_t xs = f2_fma(f2_pack(__uint_as_float(r[k2]), __uint_as_float(r[k2 + 1])), sl2, negm);
+                float x0, x1;
+                f2_unpack(xs, x0, x1);
+                const uint64_t pe = f2_pack(ex2_approx(x0), ex2_approx(x1));
+                acc2[e & 1] = f2_add(acc2[e & 1], pe);
+                float p0, p1;
+                f2_unpack(pe, p0, p1);
+                w[e] = pack_bf16x2(p0, p1);
+              }
+              tmem_st16(tm_s + wg * 32 + c * 16, w);
+            }
+            const uint64_t s01 = f2_add(acc2[0], acc2[1]);
+            float s0, s1;
+            f2_unpack(s01, s0, s1);
+            return s0 + s1;
+          };
+          // lazy rescaling: m moves only when the tile's row maximum exceeds it
+          // by more than the threshold (P stays below 2^8)
+          xput(mloc);
+          const float m_tile = fmaxf(mloc, xtake()) * p.scale_log2;
+          const bool grow = m_tile > m[ti] + kRescaleThreshold;
+          const bool resc = !first[ti] && __any_sync(0xffffffffu, grow);
+          const float factor = (grow && !first[ti]) ? ex2_approx(m[ti] - m_tile) : 1.0f;
+          if (grow) {
+            l[ti] *= factor;
+            m[ti] = m_tile;
           }
+          const float psum = make_p(m[ti]);
+          if (resc) rescale_o(factor);
+          l[ti] += psum;
           tmem_wait_st();
           tc_fence_before();
           mbar_arrive(&bars->p_full[ti]);
@@ -450,7 +475,8 @@ __global__ void __launch_bounds__(384, 1)
         mbar_wait(&bars->o_full[ti], icnt[ti] & 1, abort_flag);
         __syncwarp();
         tc_fence_after();
-        const float lt = l[ti] + exchange(l[ti]);
+        xput(l[ti]);
+        const float lt = l[ti] + xtake();
         const float inv_l = lt > 0.f ? 1.0f / lt : 0.f;
         const int a = (2 * pr + ti) * 128 + row;
         __nv_bfloat16* orow = p.o + static_cast<int64_t>(b) * p.o_sb + static_cast<int64_t>(h) * p.o_sh +

@@ -851,6 +851,8 @@ radial_status radial_device_status(void* stream) {
     RADIAL_CUDA(cudaMemcpyToSymbol(g_device_error, &zero, sizeof(int)));
     if (flag == kErrBounds)
       return fail(RADIAL_EDEVICE, "a kernel read an out-of-range index from the mask's arrays (code %d)", flag);
+    if (flag == kErrLayout)
+      return fail(RADIAL_EDEVICE, "a kernel found its dynamic shared memory misaligned and did nothing (code %d)", flag);
     return fail(RADIAL_EDEVICE, "a kernel aborted after a bounded wait ran out (code %d)", flag);
   }
   RADIAL_CUDA(cudaGetLastError());

@@ -22,6 +22,7 @@ enum DeviceErrorCode : int {
   kErrNone = 0,
   kErrWaitTimeout = 1,
   kErrBounds = 2,  // debug builds: an index read from the mask's arrays was out of range
+  kErrLayout = 3,  // the dynamic shared memory base was misaligned beyond a kernel's slack
 };
 
 // Debug builds (-DRADIAL_DEBUG) check every index the kernels read from the

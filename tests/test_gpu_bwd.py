@@ -64,6 +64,8 @@ SMALL = [
     (1, 2, 128, 2, 700, 128, 0, 36),
     (1, 1, 64, 1, 1, 64, 1, 37),
     (1, 2, 128, 9, 1000, 128, 1, 38),
+    (1, 1, 128, 24, 100, 128, 1, 39),   # 64 <= s < block: a tile spans up to three frames
+    (1, 2, 64, 16, 64, 128, 0, 40),     # s = 64: 64-token halves aligned to frames
 ]
 
 

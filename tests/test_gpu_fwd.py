@@ -67,6 +67,8 @@ SMALL = [
     (1, 1, 64, 1, 1, 64, 1, 17),         # a single token
     (1, 2, 128, 9, 1000, 128, 1, 18),    # frames not aligned to tiles
     (1, 1, 128, 12, 1560, 128, 1, 19),   # Wan-like frame size, 12 frames
+    (1, 1, 128, 24, 100, 128, 1, 20),    # 64 <= s < block: a tile spans up to three frames
+    (1, 2, 64, 16, 64, 128, 0, 21),      # s = 64: 64-key halves aligned to frames
 ]
 
 
