@@ -106,6 +106,14 @@ struct BwdCfg {
   static constexpr int SMEM_VEC = SMEM_STREAM + STAGES * 2 * TILE_BYTES;  // 2 x 2 x 128 floats
   static constexpr int SMEM_BAR = SMEM_VEC + 2 * 2 * 128 * 4;
   static constexpr int SMEM_BYTES = SMEM_BAR + 256 + 1024;
+  // dQ kernel: Q, dO fixed, then a K ring (read by S and, a tile later, by
+  // dQ) and a V ring (read by dP only, so its slots free a step earlier)
+  static constexpr int DQ_K_SLOTS = 3;
+  static constexpr int DQ_V_SLOTS = 2;
+  static constexpr int DQ_SMEM_K = SMEM_STREAM;
+  static constexpr int DQ_SMEM_V = DQ_SMEM_K + DQ_K_SLOTS * TILE_BYTES;
+  static constexpr int DQ_SMEM_BAR = DQ_SMEM_V + DQ_V_SLOTS * TILE_BYTES;
+  static constexpr int DQ_SMEM_BYTES = DQ_SMEM_BAR + 256 + 1024;
 };
 
 struct BwdBars {
@@ -113,6 +121,7 @@ struct BwdBars {
   uint64_t s_full, s_free, ew_full[2], mma2_done[2];
   uint64_t st_full[2], st_empty[2];
   uint64_t dp_full, p_ready[2], ds_ready[2];  // dK/dV kernel: S^T and dP^T halves of the handoff
+  uint64_t k_full[3], k_empty[3], v_full[2], v_empty[2];  // dQ kernel: the K and V rings
   uint32_t tmem_base;
   int abort;
 };
@@ -445,6 +454,12 @@ __global__ void __launch_bounds__(384, 1)
 // TMEM: S [0,128) dP [128,256) dQ [256,256+D) dS0 [384,448) dS1 [448,512).
 // Warps: 0 producer, 1 MMA, 2-3 idle, 4-7 and 8-11 the elementwise
 // warpgroups (key columns [0,64) and [64,128) of each tile).
+// Shared memory: Q and dO of the query tile, a 3-slot K ring and a 2-slot V
+// ring (224 KB at D = 128).  K(g) is read by S(g) and by dQ(g), which is
+// issued a tile later; V(g) only by dP(g), so its slot is released by the
+// commit after dP(g).  With one shared 2-stage ring the load of K/V(g + 1)
+// could start only when dQ(g - 1) completed, just before S(g + 1) needs it:
+// the MMA issuer waited about 1,200 of its 4,300 cycles per tile on it.
 template <int D>
 __global__ void __launch_bounds__(384, 1)
     radial_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -456,8 +471,9 @@ __global__ void __launch_bounds__(384, 1)
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   uint8_t* sQ = smem + C::SMEM_FIX;
   uint8_t* sdO = sQ + C::TILE_BYTES;
-  uint8_t* sK = smem + C::SMEM_STREAM;  // stage st: sK + st*2*TILE, V follows K
-  BwdBars* bars = reinterpret_cast<BwdBars*>(smem + C::SMEM_BAR);
+  uint8_t* sK = smem + C::DQ_SMEM_K;  // slot g % DQ_K_SLOTS
+  uint8_t* sV = smem + C::DQ_SMEM_V;  // slot g % DQ_V_SLOTS
+  BwdBars* bars = reinterpret_cast<BwdBars*>(smem + C::DQ_SMEM_BAR);
   volatile int* abort_flag = &bars->abort;
   constexpr uint32_t TM_S = 0, TM_DP = 128, TM_DQ = 256, TM_DS = 384;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -473,8 +489,14 @@ __global__ void __launch_bounds__(384, 1)
     for (int b = 0; b < 2; ++b) {
       mbar_init(&bars->ew_full[b], 256);
       mbar_init(&bars->mma2_done[b], 1);
-      mbar_init(&bars->st_full[b], 1);
-      mbar_init(&bars->st_empty[b], 1);
+    }
+    for (int b = 0; b < C::DQ_K_SLOTS; ++b) {
+      mbar_init(&bars->k_full[b], 1);
+      mbar_init(&bars->k_empty[b], 1);
+    }
+    for (int b = 0; b < C::DQ_V_SLOTS; ++b) {
+      mbar_init(&bars->v_full[b], 1);
+      mbar_init(&bars->v_empty[b], 1);
     }
     fence_barrier_init();
   }
@@ -503,20 +525,24 @@ __global__ void __launch_bounds__(384, 1)
         }
         for (int q = p.row_ptr[t]; q < p.row_ptr[t + 1]; ++q, ++it) {
           const int kb = RADIAL_CHECK_INDEX(p.col_idx[q], 0, p.nt);
-          const uint32_t st = it % C::STAGES, use = it / C::STAGES;
-          if (use > 0) mbar_wait(&bars->st_empty[st], (use - 1) & 1, abort_flag);
-          uint8_t* dK = sK + st * 2 * C::TILE_BYTES;
-          uint8_t* dV = dK + C::TILE_BYTES;
-          mbar_arrive_expect_tx(&bars->st_full[st], 2 * C::TILE_BYTES);
+          const uint32_t ks = it % C::DQ_K_SLOTS, ku = it / C::DQ_K_SLOTS;
+          if (ku > 0) mbar_wait(&bars->k_empty[ks], (ku - 1) & 1, abort_flag);
+          mbar_arrive_expect_tx(&bars->k_full[ks], C::TILE_BYTES);
 #pragma unroll
-          for (int x = 0; x < C::NBOX; ++x) {
-            tma_load_4d(dK + x * 16384, &tmK, &bars->st_full[st], x * 64, kb * 128, h, b);
-            tma_load_4d(dV + x * 16384, &tmV, &bars->st_full[st], x * 64, kb * 128, h, b);
-          }
+          for (int x = 0; x < C::NBOX; ++x)
+            tma_load_4d(sK + ks * C::TILE_BYTES + x * 16384, &tmK, &bars->k_full[ks], x * 64, kb * 128, h, b);
+          const uint32_t vs = it % C::DQ_V_SLOTS, vu = it / C::DQ_V_SLOTS;
+          if (vu > 0) mbar_wait(&bars->v_empty[vs], (vu - 1) & 1, abort_flag);
+          mbar_arrive_expect_tx(&bars->v_full[vs], C::TILE_BYTES);
+#pragma unroll
+          for (int x = 0; x < C::NBOX; ++x)
+            tma_load_4d(sV + vs * C::TILE_BYTES + x * 16384, &tmV, &bars->v_full[vs], x * 64, kb * 128, h, b);
         }
       }
-      for (uint32_t k = (it > C::STAGES ? it - C::STAGES : 0); k < it; ++k)
-        mbar_wait_drain(&bars->st_full[k % C::STAGES], (k / C::STAGES) & 1);
+      for (uint32_t k = (it > C::DQ_K_SLOTS ? it - C::DQ_K_SLOTS : 0); k < it; ++k)
+        mbar_wait_drain(&bars->k_full[k % C::DQ_K_SLOTS], (k / C::DQ_K_SLOTS) & 1);
+      for (uint32_t k = (it > C::DQ_V_SLOTS ? it - C::DQ_V_SLOTS : 0); k < it; ++k)
+        mbar_wait_drain(&bars->v_full[k % C::DQ_V_SLOTS], (k / C::DQ_V_SLOTS) & 1);
     }
   } else if (warp == 1) {
     if (lane == 0) {
@@ -525,21 +551,22 @@ __global__ void __launch_bounds__(384, 1)
       constexpr uint64_t kTile = C::TILE_BYTES >> 4;
       const uint64_t dQ = smem_desc(smem_u32(sQ), 16, 1024, kSwizzle128B);
       const uint64_t dO = smem_desc(smem_u32(sdO), 16, 1024, kSwizzle128B);
-      const uint64_t dKk = smem_desc(smem_u32(sK), 16, 1024, kSwizzle128B);       // K, V as K-major B
+      const uint64_t dKk = smem_desc(smem_u32(sK), 16, 1024, kSwizzle128B);       // K as K-major B
+      const uint64_t dVk = smem_desc(smem_u32(sV), 16, 1024, kSwizzle128B);       // V as K-major B
       const uint64_t dKmn = smem_desc(smem_u32(sK), 16384, 1024, kSwizzle128B);   // K as MN-major B
       uint32_t it = 0, item_i = 0;
       auto issue_dq = [&](uint32_t g, uint32_t j) {
-        const uint32_t st = g % C::STAGES, db = g & 1;
+        const uint32_t ks = g % C::DQ_K_SLOTS, db = g & 1;
         mbar_wait(&bars->ew_full[db], (g >> 1) & 1, abort_flag);
         if (j == 0 && item_i > 0) mbar_wait(&bars->acc_empty, (item_i - 1) & 1, abort_flag);
         tc_fence_after();
-        const uint64_t kmn = dKmn + st * 2 * kTile;
+        const uint64_t kmn = dKmn + ks * kTile;
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
           mma_ts(tmem + TM_DQ, tmem + TM_DS + db * 64 + kk * 8, kmn + kk * (2048 >> 4), idesc_g,
                  (j > 0 || kk > 0) ? 1u : 0u);
         mma_commit(&bars->mma2_done[db]);
-        mma_commit(&bars->st_empty[st]);
+        mma_commit(&bars->k_empty[ks]);
       };
       for (int item = blockIdx.x; item < p.items; item += gridDim.x, ++item_i) {
         const int bh = item / p.nt;
@@ -548,11 +575,12 @@ __global__ void __launch_bounds__(384, 1)
         mbar_wait(&bars->fix_full, item_i & 1, abort_flag);
         tc_fence_after();
         for (uint32_t j = 0; j < n_tiles; ++j) {
-          const uint32_t g = it + j, st = g % C::STAGES;
-          mbar_wait(&bars->st_full[st], (g / C::STAGES) & 1, abort_flag);
+          const uint32_t g = it + j, ks = g % C::DQ_K_SLOTS, vs = g % C::DQ_V_SLOTS;
+          mbar_wait(&bars->k_full[ks], (g / C::DQ_K_SLOTS) & 1, abort_flag);
+          mbar_wait(&bars->v_full[vs], (g / C::DQ_V_SLOTS) & 1, abort_flag);
           if (g >= 1) mbar_wait(&bars->s_free, (g - 1) & 1, abort_flag);
           tc_fence_after();
-          const uint64_t kk_ = dKk + st * 2 * kTile, vk = kk_ + kTile;
+          const uint64_t kk_ = dKk + ks * kTile, vk = dVk + vs * kTile;
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
             const uint64_t off = static_cast<uint64_t>(((kk >> 2) * 16384 + (kk & 3) * 32) >> 4);
@@ -564,6 +592,7 @@ __global__ void __launch_bounds__(384, 1)
             mma_ss(tmem + TM_DP, dO + off, vk + off, idesc_s, kk > 0 ? 1u : 0u);
           }
           mma_commit(&bars->s_full);
+          mma_commit(&bars->v_empty[vs]);  // dP(g) has read V(g)
           if (j + 1 == n_tiles) mma_commit(&bars->fix_empty);
           if (j > 0) issue_dq(g - 1, j - 1);
         }

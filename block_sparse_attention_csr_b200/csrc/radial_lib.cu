@@ -561,9 +561,9 @@ radial_status launch_bwd(const radial_csr* c, const radial_desc* d, const void* 
   if ((rs = make_bhnd_map(&mk, k, *d)) != RADIAL_OK) return rs;
   if ((rs = make_bhnd_map(&mv, v, *d)) != RADIAL_OK) return rs;
   if ((rs = make_bhnd_map(&mdo, dout, *d)) != RADIAL_OK) return rs;
-  const int smem = BwdCfg<D>::SMEM_BYTES;
+  const int smem = BwdCfg<D>::SMEM_BYTES, smem_dq = BwdCfg<D>::DQ_SMEM_BYTES;
   RADIAL_CUDA(cudaFuncSetAttribute(radial_bwd_dkdv_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
-  RADIAL_CUDA(cudaFuncSetAttribute(radial_bwd_dq_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
+  RADIAL_CUDA(cudaFuncSetAttribute(radial_bwd_dq_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_dq));
   const int64_t rows = static_cast<int64_t>(d->batch) * d->heads * d->n_tokens;
   {
     const int threads = 256;
@@ -604,7 +604,7 @@ radial_status launch_bwd(const radial_csr* c, const radial_desc* d, const void* 
   const int grid = p.items < sm_count() ? p.items : sm_count();
   radial_bwd_dkdv_kernel<D><<<grid, 384, smem, st>>>(mq, mk, mv, mdo, p);
   RADIAL_LAUNCHED();
-  radial_bwd_dq_kernel<D><<<grid, 384, smem, st>>>(mq, mk, mv, mdo, p);
+  radial_bwd_dq_kernel<D><<<grid, 384, smem_dq, st>>>(mq, mk, mv, mdo, p);
   RADIAL_LAUNCHED();
   return RADIAL_OK;
 }
