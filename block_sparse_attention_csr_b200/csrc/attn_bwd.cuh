@@ -317,6 +317,7 @@ __global__ void __launch_bounds__(384, 1)
       mg.sink = p.sink;
       mg.hd = p.hd;
       mg.cd = p.cd;
+      set_divisor(mg);
       const int c0 = p.col_ptr[u];
       const uint32_t n_tiles = static_cast<uint32_t>(p.col_ptr[u + 1] - c0);
       const float* lse_bh = p.lse + static_cast<int64_t>(bh) * p.n;
@@ -624,6 +625,7 @@ __global__ void __launch_bounds__(384, 1)
       mg.sink = p.sink;
       mg.hd = p.hd;
       mg.cd = p.cd;
+      set_divisor(mg);
       const float lse2 = valid ? p.lse[static_cast<int64_t>(bh) * p.n + a] * kLog2e : INFINITY;
       const float drow = valid ? p.dr[static_cast<int64_t>(bh) * p.n + a] : 0.f;
       const int p0 = p.row_ptr[t];

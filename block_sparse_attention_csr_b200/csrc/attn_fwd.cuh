@@ -27,15 +27,26 @@ struct RowMaskGeom {
   int32_t f, s, n, sink;
   const int32_t* hd;
   const int32_t* cd;
+  uint32_t s_mul;  // floor(x / s) = (x * s_mul) >> s_shift, set by set_divisor
+  int32_t s_shift;
 };
 
-// floor(x / s) for 0 <= x < 2^30 without an integer division: a float
-// estimate from the reciprocal, then an exact correction of at most one step.
-__device__ __forceinline__ int div_by(int x, int s) {
-  int q = __float2int_rz(static_cast<float>(x) * __frcp_rn(static_cast<float>(s)));
-  q += (q + 1) * s <= x;
-  q -= q * s > x;
-  return q;
+// Exact division by the frame size with one multiply and one shift
+// (Granlund and Montgomery, "Division by invariant integers using
+// multiplication", 1994, Thm 4.2 with N = 31): with l = ceil(log2 s) and
+// m = ceil(2^(31+l) / s) < 2^32, floor(x / s) = floor(x m / 2^(31+l)) for every
+// 0 <= x < 2^31.  Computed once per thread; the per-tile divisions then stay
+// off the exponential unit (an integer divide or a float reciprocal would
+// issue there).
+__device__ __forceinline__ void set_divisor(RowMaskGeom& p) {
+  int l = 0;
+  while (l < 31 && (1u << l) < static_cast<uint32_t>(p.s)) ++l;
+  const uint64_t num = (uint64_t(1) << (31 + l)) + static_cast<uint64_t>(p.s) - 1;
+  p.s_mul = static_cast<uint32_t>(num / static_cast<uint64_t>(p.s));
+  p.s_shift = 31 + l;
+}
+__device__ __forceinline__ int div_s(const RowMaskGeom& p, int x) {
+  return static_cast<int>((static_cast<uint64_t>(static_cast<uint32_t>(x)) * p.s_mul) >> p.s_shift);
 }
 
 // Bits [lo, hi] of a 64-bit word, 0 <= lo <= hi <= 63.
@@ -78,7 +89,7 @@ __device__ __forceinline__ uint64_t window_mask64(const RowMaskGeom& p, int own,
     if (!kKeys && p.sink && j == 0) return bit_range64(lo_s, hi_s);
     return interval_bits64(p, own, pos, b0, j, lo_s, hi_s);
   };
-  int j = div_by(b0, p.s);
+  int j = div_s(p, b0);
   if (p.s >= 64) {
     const int e = (j + 1) * p.s - b0;  // first column of frame j + 1
     if (e >= bend) return seg(j, 0, bend - 1);

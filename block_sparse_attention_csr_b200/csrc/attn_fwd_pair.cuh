@@ -326,6 +326,7 @@ __global__ void __launch_bounds__(384, 1)
     mp.sink = p.sink;
     mp.hd = p.hd;
     mp.cd = p.cd;
+    set_divisor(mp);
     uint32_t g[2] = {0u, 0u}, icnt[2] = {0u, 0u};
     for (int item = blockIdx.x; item < p.items; item += gridDim.x) {
       const int bh = item / p.np;

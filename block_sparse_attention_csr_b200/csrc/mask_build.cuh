@@ -36,14 +36,26 @@ struct MaskGeom {
 
 // h(d) and c(d): the closed form r = floor(log2 max(d,1)), h = floor(s/2^r)-1,
 // c = ceil(2^r/s), or the table of an ablation mask.
+// floor(log2 d) for d >= 1 by shifts and compares.  The attention kernels
+// evaluate it per PARTIAL tile next to a stream of exponentials; a count of
+// leading zeros (like a conversion or a reciprocal) issues at the exponential
+// unit's rate of 16 per clock and SM and would queue behind them.
+__device__ __forceinline__ int floor_log2(int d) {
+  int r = 0;
+  if (d >> 16) { d >>= 16; r += 16; }
+  if (d >> 8) { d >>= 8; r += 8; }
+  if (d >> 4) { d >>= 4; r += 4; }
+  if (d >> 2) { d >>= 2; r += 2; }
+  return r + (d >> 1);
+}
 __device__ __forceinline__ int half_width_of(const int32_t* hd, int s, int d) {
   if (hd) return hd[d];
-  const int r = 31 - __clz(d > 1 ? d : 1);
+  const int r = floor_log2(d > 1 ? d : 1);
   return (s >> r) - 1;
 }
 __device__ __forceinline__ long long period_of(const int32_t* cd, int s, int d) {
   if (cd) return cd[d];
-  const int r = 31 - __clz(d > 1 ? d : 1);
+  const int r = floor_log2(d > 1 ? d : 1);
   return ((1LL << r) + s - 1) / s;
 }
 
