@@ -49,7 +49,9 @@ typedef enum radial_status {
   RADIAL_ECUDA = 4,         /* a CUDA runtime or driver call failed */
   RADIAL_EDEVICE = 5        /* a kernel aborted after a bounded wait ran out (or, in
                                the bounds-checking debug build, read an out-of-range
-                               index from the mask's arrays) */
+                               index from the mask's arrays; or found its dynamic
+                               shared memory too misaligned for its layout and did
+                               nothing) */
 } radial_status;
 
 /* Mask parameters.  sink: 1 = every query also attends to all tokens of frame
