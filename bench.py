@@ -63,6 +63,36 @@ def tile_flops(wl, nnz, backward=False, heads=None):
     return per * wl.block * wl.block * wl.head_dim * nnz * wl.batch * heads
 
 
+def allowed_pairs(frames, s, sink=True):
+    """Allowed (query, key) token pairs of one head under the method's mask, by
+    frame pair: the sink frame whole (s^2); a band |k - l| <= h clipped to the
+    frame, s(2h+1) - h(h+1) pairs (s^2 once h >= s - 1); a sampled diagonal, s
+    pairs when d is a multiple of its period c; none otherwise.  h = floor(s /
+    2^r) - 1 and c = ceil(2^r / s) with r = floor(log2 max(d, 1)) (the review
+    page, Sec. 4.2: Eq.4 and Fig.5)."""
+    by_d = {}
+    for d in range(frames):
+        r = max(d, 1).bit_length() - 1
+        h = (s >> r) - 1
+        if h >= 0:
+            hh = min(h, s - 1)
+            by_d[d] = s * (2 * hh + 1) - hh * (hh + 1)
+        else:
+            c = -(-(1 << r) // s)
+            by_d[d] = s if d % c == 0 else 0
+    total = 0
+    for i in range(frames):
+        for j in range(frames):
+            total += s * s if (sink and j == 0) else by_d[abs(i - j)]
+    return total
+
+
+def elem_flops(wl, pairs, heads=None):
+    """Algorithmic forward flops on allowed element pairs only: 4*d per pair."""
+    heads = wl.heads if heads is None else heads
+    return 4 * wl.head_dim * pairs * wl.batch * heads
+
+
 def whole_job_tflops(flops_per_rank, world, ms_max):
     """Whole-job throughput: every rank runs one replica of the workload
     (independent problems), so the job does world * flops_per_rank in the
@@ -416,6 +446,7 @@ def run_ours(args, rank, world, local_rank):
         cpu = cpu_baseline(wl, nnz, q, k, v, budget_s=args.cpu_budget, backward=backward)
 
     if rank == 0:
+        pairs = allowed_pairs(wl.frames, wl.tokens_per_frame, sink=True)
         traffic = None
         tp = os.path.join(ROOT, "profiles", "fwd_traffic.json")
         if os.path.exists(tp):
@@ -440,6 +471,11 @@ def run_ours(args, rank, world, local_rank):
                          "unit": "TFLOP/s", "frac": fwd_tf / peak, "peak_source": f"{peak_src} bf16 burst",
                          "frac_of_sustained": fwd_tf / peak_sus, "traffic": traffic,
                          "algorithmic_flops_per_launch": tile_flops(wl, nnz, heads=local_heads), "launch_ms": fwd_ms},
+            "elem": {"allowed_pairs_per_head": pairs, "flops_per_launch": elem_flops(wl, pairs, heads=local_heads),
+                     "achieved": elem_flops(wl, pairs, heads=local_heads) / (fwd_ms * 1e-3) / 1e12,
+                     "frac": elem_flops(wl, pairs, heads=local_heads) / (fwd_ms * 1e-3) / 1e12 / peak,
+                     "note": "forward flops on allowed token pairs only (4*d per pair); the tile figure above "
+                             "also counts the masked lanes of PARTIAL tiles"},
             "cpu_baseline": cpu,
             "e2e": e2e,
             "gpu_launches": int(launches),
