@@ -745,10 +745,31 @@ extern "C" radial_status radial_attn_fwd_staged(const radial_csr* c, const radia
   RADIAL_CUDA(cudaEventRecord(R->start, st));
   RADIAL_CUDA(cudaStreamWaitEvent(R->in, R->start, 0));
   RADIAL_CUDA(cudaStreamWaitEvent(R->out, R->start, 0));
+  // Head groups of one batch entry.  The first group's copy-in and the last
+  // group's copy-out overlap no attention, so with three or more groups those
+  // two are small and the groups between them grow: weights 1, 2, 4, 4, ...,
+  // 4 and 1 for the last, rounded to whole heads with at least one per group.
+  std::vector<int> bound(per_b + 1, 0);
+  {
+    std::vector<int64_t> cw(per_b);
+    int64_t W = 0;
+    for (int k = 0; k < per_b; ++k) {
+      const int64_t w = (per_b <= 2 || k == per_b - 1) ? 1 : (int64_t(1) << std::min(k, 2));
+      W += w;
+      cw[k] = W;
+    }
+    for (int k = 0; k < per_b; ++k) {
+      int x = static_cast<int>((static_cast<int64_t>(d->heads) * cw[k] + W / 2) / W);
+      x = std::max(x, bound[k] + 1);
+      x = std::min(x, d->heads - (per_b - 1 - k));
+      bound[k + 1] = x;
+    }
+    bound[per_b] = d->heads;
+  }
   int g = 0;
   for (int b = 0; b < d->batch; ++b) {
     for (int k = 0; k < per_b; ++k, ++g) {
-      const int h0 = k * d->heads / per_b, h1 = (k + 1) * d->heads / per_b;
+      const int h0 = bound[k], h1 = bound[k + 1];
       // copy in
       if ((rs = copy_heads(q_dev, q_host, *d, b, h0, h1, cudaMemcpyHostToDevice, R->in)) != RADIAL_OK) return rs;
       if ((rs = copy_heads(k_dev, k_host, *d, b, h0, h1, cudaMemcpyHostToDevice, R->in)) != RADIAL_OK) return rs;

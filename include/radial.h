@@ -169,7 +169,11 @@ radial_status radial_attn_fwd(const radial_csr* csr, const radial_desc* desc, co
  * O and LSE back, but the heads of each batch entry are processed in `chunks`
  * groups (at most batch * chunks = 64 groups), and group g's inputs are copied
  * in while group g-1 is computed and group g-1's outputs copied out, on two
- * internal streams per device created on the first call.  q_host .. lse_host
+ * internal streams per device created on the first call.  The first group's
+ * copy-in and the last group's copy-out overlap no attention, so with three
+ * or more groups their sizes follow the weights 1, 2, 4, 4, ..., 4 and 1 for
+ * the last group (each group at least one head); one or two groups split the
+ * heads evenly.  q_host .. lse_host
  * are host buffers, q_dev .. lse_dev caller-owned device buffers of the full
  * shape; host and device tensors share the layout of `desc`.  The host
  * buffers should be page-locked, or the copies cannot overlap.  Work already

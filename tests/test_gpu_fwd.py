@@ -170,7 +170,7 @@ def test_many_work_items_all_rows():
            np.concatenate([a for a, _ in res]), np.concatenate([b for _, b in res]), "many items")
 
 
-@pytest.mark.parametrize("Bn,H,chunks,permuted", [(1, 5, 3, False), (2, 4, 4, False), (1, 6, 2, True)])
+@pytest.mark.parametrize("Bn,H,chunks,permuted", [(1, 5, 3, False), (2, 4, 4, False), (1, 6, 2, True), (1, 8, 6, False)])
 def test_staged_forward_equals_device_forward(Bn, H, chunks, permuted):
     """radial_attn_fwd_staged (host buffers, copies overlapped with the
     attention group by group) gives bit for bit the device call's O and LSE:
