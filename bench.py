@@ -620,7 +620,7 @@ def run_reference(args, rank, world):
               f"{wl.batch * wl.heads * wl.n} rows" + (" x3.5 for forward+backward" if wl.backward else ""))
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": full_s * 1e3, "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "scaling": "strong" if heads_mode else "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": dict(config_of(wl, nnz), parallelism=(f"heads/{world}" if heads_mode else f"replica x{world}"),
                            heads_per_rank_max=-(-wl.heads // world) if heads_mode else wl.heads),
             "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": _cores(), "kind": "oracle", "sample": sample},
