@@ -376,7 +376,7 @@ def run_ours(args, rank, world, local_rank):
                             "note": "10*B^2*d flops per tile (5 GEMMs); the kernels issue 7 (dQ pass recomputes S, dP)"}
             del dq, dk, dv, ws
 
-    if rank == 0 and args.sweep:
+    if rank == 0 and (args.sweep or (args.sweep is None and world == 1 and not args.quick and args.workload == "hunyuan720p")):
         extra["sweep"] = run_sweep(args, dev, stream, peak)
 
     if rank == 0 and args.lora:
@@ -640,7 +640,9 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--ref-rows", type=int, default=512)
-    ap.add_argument("--sweep", action="store_true", help="add the frame-count scaling sweep (radial vs dense)")
+    ap.add_argument("--sweep", action="store_true", default=None,
+                    help="add the frame-count scaling sweep (radial vs dense); on by default on one GPU")
+    ap.add_argument("--no-sweep", dest="sweep", action="store_false")
     ap.add_argument("--lora", action="store_true", help="add one LoRA-adapted attention layer step (fwd+bwd)")
     ap.add_argument("--lora-rank", type=int, default=64)
     ap.add_argument("--step", default=None, choices=["fwd", "bwd", "fwdbwd"],
