@@ -10,7 +10,7 @@
 // shifted by 128 tokens); a key tile only one of them needs is computed for
 // that tile alone.
 //
-// Warp roles (384 threads; at most 168 registers each, 144 used):
+// Warp roles (384 threads; at most 168 registers each, 127 used):
 //   warp 0      TMA producer: Q0, Q1 once per item; K and V through
 //               separate 3-slot / 2-slot rings, K one union column ahead of V.
 //   warps 2-3   idle (keep the softmax warps on warpgroup boundaries).
@@ -95,12 +95,13 @@ struct FwdPairCfg {
 
 struct PairBars {
   uint64_t q_full, q_empty, mma_done;
-  uint64_t k_full[3], k_empty[3], v_full[2], v_empty[2];
+  uint64_t k_full[3], k_empty[3], v_full[3], v_empty[3];
   uint64_t s_full[2], p_full[2], o_full[2], o_empty[2];
   uint32_t tmem_base;
   int abort;
 };
 static_assert(sizeof(PairBars) <= 256, "barriers overlap the row exchange buffer");
+static_assert(FwdPairCfg<128>::K_SLOTS <= 3 && FwdPairCfg<128>::V_SLOTS <= 3, "ring barriers hold 3 slots");
 
 template <int D>
 __global__ void __launch_bounds__(384, 1)
@@ -130,9 +131,11 @@ __global__ void __launch_bounds__(384, 1)
       mbar_init(&bars->k_full[i], 1);
       mbar_init(&bars->k_empty[i], 1);
     }
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < C::V_SLOTS; ++i) {
       mbar_init(&bars->v_full[i], 1);
       mbar_init(&bars->v_empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
       mbar_init(&bars->s_full[i], 1);
       mbar_init(&bars->p_full[i], 256);
       mbar_init(&bars->o_full[i], 1);
@@ -166,7 +169,7 @@ __global__ void __launch_bounds__(384, 1)
         ++kc;
       };
       auto load_v = [&](int kb, int h, int b) {
-        const uint32_t sl = vc & 1, use = vc >> 1;
+        const uint32_t sl = vc % C::V_SLOTS, use = vc / C::V_SLOTS;
         if (use > 0) mbar_wait(&bars->v_empty[sl], (use - 1) & 1, abort_flag);
         mbar_arrive_expect_tx(&bars->v_full[sl], C::TILE_BYTES);
 #pragma unroll
@@ -195,7 +198,8 @@ __global__ void __launch_bounds__(384, 1)
       }
       for (uint32_t x = (kc > C::K_SLOTS ? kc - C::K_SLOTS : 0); x < kc; ++x)
         mbar_wait_drain(&bars->k_full[x % C::K_SLOTS], (x / C::K_SLOTS) & 1);
-      for (uint32_t x = (vc > 2 ? vc - 2 : 0); x < vc; ++x) mbar_wait_drain(&bars->v_full[x & 1], (x >> 1) & 1);
+      for (uint32_t x = (vc > C::V_SLOTS ? vc - C::V_SLOTS : 0); x < vc; ++x)
+        mbar_wait_drain(&bars->v_full[x % C::V_SLOTS], (x / C::V_SLOTS) & 1);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
@@ -228,8 +232,8 @@ __global__ void __launch_bounds__(384, 1)
         auto issue_pv = [&](int i, uint32_t vslot_count) {
           const uint32_t gi = pend_g[i];
           mbar_wait(&bars->p_full[i], gi & 1, abort_flag);
-          const uint32_t vs = vslot_count & 1;
-          mbar_wait(&bars->v_full[vs], (vslot_count >> 1) & 1, abort_flag);
+          const uint32_t vs = vslot_count % C::V_SLOTS;
+          mbar_wait(&bars->v_full[vs], (vslot_count / C::V_SLOTS) & 1, abort_flag);
           if (first_pv[i] && icnt[i] > 0) mbar_wait(&bars->o_empty[i], (icnt[i] - 1) & 1, abort_flag);
           tc_fence_after();
           const uint64_t dv = dv0 + vs * kSlot;
@@ -269,7 +273,7 @@ __global__ void __launch_bounds__(384, 1)
           }
           mma_commit(&bars->k_empty[ks]);  // K(u) read by the S MMAs above
           ++kc;
-          if (u > u0) mma_commit(&bars->v_empty[(vc - 1) & 1]);  // V(u-1): its PVs are issued
+          if (u > u0) mma_commit(&bars->v_empty[(vc - 1) % C::V_SLOTS]);  // V(u-1): its PVs are issued
           if (u + 1 == u1) mma_commit(&bars->q_empty);
           ++vc;  // V(u) is the producer's next V; PVs of column u refer to vc - 1
         }
@@ -277,7 +281,7 @@ __global__ void __launch_bounds__(384, 1)
 #pragma unroll
         for (int i = 0; i < 2; ++i)
           if (pending[i]) issue_pv(i, vc - 1);
-        mma_commit(&bars->v_empty[(vc - 1) & 1]);
+        mma_commit(&bars->v_empty[(vc - 1) % C::V_SLOTS]);
 #pragma unroll
         for (int i = 0; i < 2; ++i)
           if (used[i]) {
@@ -357,14 +361,9 @@ __global__ void __launch_bounds__(384, 1)
 #pragma unroll
         for (int ti = 0; ti < 2; ++ti) {
           if (!(fl & (ti == 0 ? kPairIn0 : kPairIn1))) continue;
-          mbar_wait(&bars->s_full[ti], g[ti] & 1, abort_flag);
-          __syncwarp();
-          tc_fence_after();
-          const uint32_t tm_s = tmem + lane_addr + C::TM_S + ti * 128;
-          uint32_t r[64];
-          tmem_ld32(tm_s + col0, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
-          tmem_ld32(tm_s + col0 + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
-          // the mask bits of a PARTIAL tile are computed while the load is in flight
+          // The mask bits of a PARTIAL tile depend only on the key tile and the
+          // row: they are formed before the wait for S, which they mostly fill
+          // (PARTIAL tiles tend to wait longest on the MMA chain).
           const bool part = (fl & (ti == 0 ? kPairPart0 : kPairPart1)) != 0;
           uint32_t mw[2] = {0xffffffffu, 0xffffffffu};
           if (part) {
@@ -381,6 +380,13 @@ __global__ void __launch_bounds__(384, 1)
               else if (!__all_sync(0xffffffffu, mw[c] == 0xffffffffu)) mixed |= 1u << c;
             }
           }
+          mbar_wait(&bars->s_full[ti], g[ti] & 1, abort_flag);
+          __syncwarp();
+          tc_fence_after();
+          const uint32_t tm_s = tmem + lane_addr + C::TM_S + ti * 128;
+          uint32_t r[64];
+          tmem_ld32(tm_s + col0, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
+          tmem_ld32(tm_s + col0 + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
           tmem_wait_ld();
           float acc[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
