@@ -496,7 +496,8 @@ def run_sweep(args, dev, stream, peak):
     from block_sparse_attention_csr_b200 import inputs as I
 
     def timed(csr, q, k, v, o, lse, reps):
-        rb.radial_attn_fwd(csr, q, k, v, o=o, lse=lse, stream=stream)
+        for _ in range(3):  # warm-up
+            rb.radial_attn_fwd(csr, q, k, v, o=o, lse=lse, stream=stream)
         ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(reps)]
         for a, b in ev:
             a.record(stream)
