@@ -378,6 +378,7 @@ def run_ours(args, rank, world, local_rank):
 
     if rank == 0 and (args.sweep or (args.sweep is None and world == 1 and not args.quick and args.workload == "hunyuan720p")):
         extra["sweep"] = run_sweep(args, dev, stream, peak)
+        extra["long_step"] = run_long_step(dev, stream, peak)
 
     if rank == 0 and args.lora:
         extra["lora_layer"] = run_lora_layer(wl, csr, dev, stream, args.lora_rank)
@@ -525,6 +526,47 @@ def run_sweep(args, dev, stream, peak):
                     "dense_tflops": tile_flops(wl, dnnz) / (dms * 1e-3) / 1e12, "speedup_vs_dense": dms / ms})
         del q, k, v, o, lse, csr, dcsr
         torch.cuda.empty_cache()
+    return out
+
+
+def run_long_step(dev, stream, peak):
+    """The 4x-length step's attention (132 frames x 3600 tokens, 24 heads, d 128:
+    the shape the length-extension fine-tuning runs at): forward and backward
+    times, median of three after one warm-up."""
+    import numpy as np
+    import torch
+    import block_sparse_attention_csr_b200 as rb
+    from block_sparse_attention_csr_b200 import inputs as I
+
+    wl = I.WORKLOADS["hunyuan720p_4x"]
+    q, k, v, do = I.draw(wl, device=dev, backward=True)
+    o = torch.empty_like(q)
+    lse = torch.empty(q.shape[:3], dtype=torch.float32, device=dev)
+    dq, dk, dv = (torch.empty_like(q) for _ in range(3))
+    ws = torch.empty(max(256, rb.radial_attn_bwd_workspace_size(q)), dtype=torch.uint8, device=dev)
+    csr = rb.radial_mask_build(wl.frames, wl.tokens_per_frame, wl.block, sink=1)
+    nnz = rb.radial_csr_info(csr)["nnz"]
+
+    def timed(fn, reps=3):
+        fn()
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(reps)]
+        for a, b in ev:
+            a.record(stream)
+            fn()
+            b.record(stream)
+        torch.cuda.synchronize(dev)
+        return float(np.median([a.elapsed_time(b) for a, b in ev]))
+
+    fwd_ms = timed(lambda: rb.radial_attn_fwd(csr, q, k, v, o=o, lse=lse, stream=stream))
+    bwd_ms = timed(lambda: rb.radial_attn_bwd(csr, do, q, k, v, o, lse, dq, dk, dv, ws, stream=stream))
+    rb.radial_device_status(stream)
+    out = {"workload": wl.name, "active_tiles": int(nnz), "fwd_ms": fwd_ms, "bwd_ms": bwd_ms,
+           "step_ms": fwd_ms + bwd_ms,
+           "fwd_tflops": tile_flops(wl, nnz) / (fwd_ms * 1e-3) / 1e12,
+           "bwd_tflops_algorithmic": tile_flops(wl, nnz, True) / (bwd_ms * 1e-3) / 1e12,
+           "fwd_pct_of_peak": 100 * tile_flops(wl, nnz) / (fwd_ms * 1e-3) / 1e12 / peak}
+    del q, k, v, do, o, lse, dq, dk, dv, ws, csr
+    torch.cuda.empty_cache()
     return out
 
 
