@@ -235,18 +235,44 @@ __global__ void __launch_bounds__(256, 1)
 }
 
 // out[c, r] = in[r, c] for a bf16 [R, Cc] matrix (row strides in elements).
-__global__ void transpose_bf16_kernel(const __nv_bfloat16* __restrict__ in, int64_t ld_in, int R, int Cc,
-                                      __nv_bfloat16* __restrict__ out, int64_t ld_out) {
-  __shared__ __nv_bfloat16 tile[32][33];
-  const int c0 = blockIdx.x * 32, r0 = blockIdx.y * 32;
-  for (int y = threadIdx.y; y < 32; y += blockDim.y) {
-    const int r = r0 + y, c = c0 + threadIdx.x;
-    if (r < R && c < Cc) tile[y][threadIdx.x] = in[static_cast<int64_t>(r) * ld_in + c];
+__global__ void __launch_bounds__(256) transpose_bf16_kernel(const __nv_bfloat16* __restrict__ in, int64_t ld_in,
+                                                            int R, int Cc, __nv_bfloat16* __restrict__ out,
+                                                            int64_t ld_out) {
+  // 64 x 64 tiles moved as bf16 pairs: every warp access is a whole 128-byte
+  // line.  Rows of 66 bf16 (33 words) keep the column reads at two-way bank
+  // conflicts.  Pairs need even column offsets, which the callers' leading
+  // dimensions and column counts (multiples of 8) give; ragged edges fall
+  // back to single elements.
+  __shared__ __align__(16) __nv_bfloat16 tile[64][66];
+  const int c0 = blockIdx.x * 64, r0 = blockIdx.y * 64;
+  const int tx = threadIdx.x, ty = threadIdx.y;  // 32 x 8
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    const int y = ty + 8 * k, r = r0 + y, c = c0 + 2 * tx;
+    if (r < R) {
+      const __nv_bfloat16* src = in + static_cast<int64_t>(r) * ld_in + c;
+      if (c + 1 < Cc) {
+        *reinterpret_cast<__nv_bfloat162*>(&tile[y][2 * tx]) = *reinterpret_cast<const __nv_bfloat162*>(src);
+      } else if (c < Cc) {
+        tile[y][2 * tx] = src[0];
+      }
+    }
   }
   __syncthreads();
-  for (int y = threadIdx.y; y < 32; y += blockDim.y) {
-    const int c = c0 + y, r = r0 + threadIdx.x;
-    if (c < Cc && r < R) out[static_cast<int64_t>(c) * ld_out + r] = tile[threadIdx.x][y];
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    const int y = ty + 8 * k, c = c0 + y, r = r0 + 2 * tx;  // output row c, output columns r, r + 1
+    if (c < Cc) {
+      __nv_bfloat16* dst = out + static_cast<int64_t>(c) * ld_out + r;
+      if (r + 1 < R) {
+        __nv_bfloat162 v;
+        v.x = tile[2 * tx][y];
+        v.y = tile[2 * tx + 1][y];
+        *reinterpret_cast<__nv_bfloat162*>(dst) = v;
+      } else if (r < R) {
+        dst[0] = tile[2 * tx][y];
+      }
+    }
   }
 }
 

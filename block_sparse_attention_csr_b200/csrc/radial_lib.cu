@@ -999,7 +999,7 @@ radial_status launch_gemm(int64_t M, int64_t N, const GemmSeg& s0, const GemmSeg
 
 radial_status launch_transpose(const void* in, int64_t ld_in, int64_t R, int64_t Cc, void* out, int64_t ld_out,
                                cudaStream_t st) {
-  dim3 grid(static_cast<unsigned>((Cc + 31) / 32), static_cast<unsigned>((R + 31) / 32));
+  dim3 grid(static_cast<unsigned>((Cc + 63) / 64), static_cast<unsigned>((R + 63) / 64));
   transpose_bf16_kernel<<<grid, dim3(32, 8), 0, st>>>(reinterpret_cast<const __nv_bfloat16*>(in), ld_in,
                                                       static_cast<int>(R), static_cast<int>(Cc),
                                                       reinterpret_cast<__nv_bfloat16*>(out), ld_out);
