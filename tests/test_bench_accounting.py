@@ -29,3 +29,16 @@ def test_hunyuan_element_flops():
     wl = I.WORKLOADS["hunyuan720p"]
     pairs = bench.allowed_pairs(wl.frames, wl.tokens_per_frame)
     assert abs(bench.elem_flops(wl, pairs) / 1e12 - 67.84) < 0.01
+
+
+def test_hunyuan_tile_flops_from_oracle_plan():
+    """Tile-level work of the bench line: 4*B^2*d flops per active 128x128 tile
+    (QK^T and PV) over the oracle's own tile classification -- 389,411 active
+    tiles per head and 78.40 TFLOP per forward launch at the HunyuanVideo shape."""
+    import numpy as np
+    from block_sparse_attention_csr_b200 import inputs as I
+    from oracle.mask import tile_states_intervals
+    wl = I.WORKLOADS["hunyuan720p"]
+    nnz = int(np.count_nonzero(tile_states_intervals(wl.frames, wl.tokens_per_frame, wl.block, True)))
+    assert nnz == 389_411
+    assert abs(bench.tile_flops(wl, nnz) / 1e12 - 78.40) < 0.01
